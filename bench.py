@@ -1,0 +1,452 @@
+"""Benchmark of the H3-style DiT attention core on B200.
+
+One step = the whole hot path over one batch of the 5 s 1344x768 clip latent
+(31x48x84 = 124,992 tokens, 56 heads x 96, bf16, structured synthetic data):
+    fused QK-RMSNorm + 3D RoPE  ->  blockwise router (sparsity 0.75)
+    ->  block-sparse attention  ->  dense attention
+The headline value is attention TFLOP/s over the whole step (algorithmic
+FLOPs of both attention passes / step time).  Per-kernel times come from CUDA
+events on the launching stream inside the timed region.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Under torchrun (N > 1) every rank runs its own clip (weak scaling, no data-path
+collective); rank 0 prints the max-over-ranks line.  --impl reference times the
+fp64 CPU oracle on a bounded sample of the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD = "video5s_sparse"
+SPARSITY = 0.75
+METRIC = "attention TFLOP/s and % of B200 bf16 peak at ~125k tokens; prologue GB/s vs HBM"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def attention_flops(N: int, heads: int, B: int, d: int = 96, blocks: np.ndarray | None = None, block: int = 128):
+    """4*d FLOPs per (query, key) pair attended: QK^T and PV, 2 FLOPs per MAC each."""
+    if blocks is None:
+        return 4.0 * d * heads * B * float(N) * float(N)
+    nblk = (N + block - 1) // block
+    lens = np.full(nblk, block, dtype=np.float64)
+    lens[-1] = N - (nblk - 1) * block
+    # sum over (b, h, i, j in list_i) of |blk_i| * |blk_j|
+    pairs = lens[blocks].sum(axis=-1)                  # [B, H, nblk]
+    return 4.0 * d * float((pairs * lens[None, None, :]).sum())
+
+
+def prologue_bytes(N: int, heads: int, B: int, d: int = 96) -> float:
+    """Read + write of Q and K in bf16: 4 bytes per element per tensor pair."""
+    return 2.0 * 2 * 2 * B * N * heads * d
+
+
+def router_bytes(N: int, heads: int, B: int, d: int = 96) -> float:
+    """The pooling pass reads Q and K once."""
+    return 2.0 * 2 * B * N * heads * d
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples during the timed region."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in getattr(self, "lines", []):
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return rank, world, local
+
+
+def allreduce_max(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def load_traffic():
+    """ncu DRAM bytes per launch, kept only while the kernel sources are unchanged."""
+    if not os.path.exists(PROFILE_TRAFFIC):
+        return {}
+    import hashlib
+
+    with open(PROFILE_TRAFFIC) as f:
+        rec = json.load(f)
+    out = {}
+    for kernel, ent in rec.items():
+        src = os.path.join(ROOT, ent["source"])
+        if os.path.exists(src) and hashlib.sha256(open(src, "rb").read()).hexdigest() == ent["sha256"]:
+            out[kernel] = ent
+    return out
+
+
+# ----------------------------------------------------------------- GPU arm
+
+def run_gpu(args, rank, world, local):
+    import rope_block_sparse_b200 as h3a
+    from rope_block_sparse_b200 import synth
+
+    w = synth.WORKLOADS[args.workload]
+    grid, heads, B, N = w.grid, w.heads, w.B, w.N
+    d = synth.draw_workload(args.workload, seed=rank)
+    dev = torch.device("cuda", local)
+    q, k, v = (d[n].to(dev) for n in "qkv")
+    gq, gk = d["gamma_q"].to(dev), d["gamma_k"].to(dev)
+    qn, kn = torch.empty_like(q), torch.empty_like(k)
+    o_dense, o_sparse = torch.empty_like(q), torch.empty_like(q)
+    nblk = (N + 127) // 128
+    kk = h3a.route_k(nblk, SPARSITY)
+    blocks = torch.empty((B, heads, nblk, kk), dtype=torch.int32, device=dev)
+    ws = torch.empty(h3a.route_workspace_size(q), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        h3a.qk_norm_rope(q, k, gq, gk, grid, out=(qn, kn))
+        if ev is not None:
+            ev[1].record(stream)
+        h3a.route(qn, kn, SPARSITY, workspace=ws, out=blocks)
+        if ev is not None:
+            ev[2].record(stream)
+        h3a.attention(qn, kn, v, blocks, out=o_sparse)
+        if ev is not None:
+            ev[3].record(stream)
+        h3a.attention(qn, kn, v, None, out=o_dense)
+        if ev is not None:
+            ev[4].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if h3a.last_device_error() != 0:
+        raise RuntimeError("device-side timeout during warm-up")
+    flops_dense = attention_flops(N, heads, B)
+    flops_sparse = attention_flops(N, heads, B, blocks=blocks.cpu().numpy())
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        for i in range(args.steps):
+            step(evs[i])
+        torch.cuda.synchronize()
+    barrier(world)
+    if h3a.last_device_error() != 0:
+        raise RuntimeError("device-side timeout in the timed region")
+    per = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(4)] for i in range(args.steps)])
+    step_ms_local = float(sum(evs[i][0].elapsed_time(evs[i][4]) for i in range(args.steps)) / args.steps)
+    step_ms = allreduce_max(step_ms_local, world)
+    kern_ms = {name: allreduce_max(float(per[:, j].mean()), world)
+               for j, name in enumerate(["prologue", "router", "attention_sparse", "attention_dense"])}
+
+    # end to end through the public API with host buffers
+    e2e = None
+    if args.e2e_steps > 0:
+        hq, hk, hv = (d[n].pin_memory() for n in "qkv")
+        hod = torch.empty(q.shape, dtype=torch.bfloat16).pin_memory()
+        hos = torch.empty(q.shape, dtype=torch.bfloat16).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
+        d2h = hod.numel() * 2 + hos.numel() * 2
+
+        def e2e_step():
+            q.copy_(hq, non_blocking=True)
+            k.copy_(hk, non_blocking=True)
+            v.copy_(hv, non_blocking=True)
+            step()
+            hos.copy_(o_sparse, non_blocking=True)
+            hod.copy_(o_dense, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier(world)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        e2e_ms = allreduce_max(e0.elapsed_time(e1) / args.e2e_steps, world)
+        e2e = {"value": round(world * (flops_dense + flops_sparse) / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 3),
+               "steps": args.e2e_steps}
+    clocks = clk.summary()
+    if rank != 0:
+        return None
+
+    pk, pk_src = peaks()
+    dense_tflops = flops_dense / (kern_ms["attention_dense"] * 1e-3) / 1e12
+    sparse_tflops = flops_sparse / (kern_ms["attention_sparse"] * 1e-3) / 1e12
+    pro_gbs = prologue_bytes(N, heads, B) / (kern_ms["prologue"] * 1e-3) / 1e9
+    router_gbs = router_bytes(N, heads, B) / (kern_ms["router"] * 1e-3) / 1e9
+    traffic = load_traffic()
+    peak_t = pk["bf16_tflops_sustained"]
+    line = {
+        "metric": METRIC,
+        "value": round(world * (flops_dense + flops_sparse) / (step_ms * 1e-3) / 1e12, 3),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(step_ms, 3),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {
+            "workload": f"{w.name}: B={B}, {heads} heads x 96, grid {grid[0]}x{grid[1]}x{grid[2]} = {N:,} tokens "
+                        f"per GPU; prologue + router (sparsity {SPARSITY}, k={kk}/{nblk}) + sparse + dense attention",
+            "tokens": N, "heads": heads, "head_dim": 96, "batch_per_gpu": B, "sparsity": SPARSITY,
+            "parallelism": f"dp{world} (independent clips per GPU)",
+            "l2": f"inputs larger than L2 (Q, K, V {B * N * heads * 96 * 2 / 1e9:.2f} GB each); no explicit flush",
+        },
+        "roofline": {
+            "kernel": "attention_kernel (dense)",
+            "bound": "tensor",
+            "achieved": round(dense_tflops, 2),
+            "peak": peak_t,
+            "unit": "TFLOP/s",
+            "frac": round(dense_tflops / peak_t, 4),
+            "peak_source": f"{pk_src} bf16 sustained (kernel timed inside a long step)",
+            "frac_of_burst": round(dense_tflops / pk["bf16_tflops"], 4),
+            "frac_of_spec_2250": round(dense_tflops / 2250.0, 4),
+            "traffic": traffic.get("attention_dense", {}).get("bytes_per_launch"),
+            "algorithmic_flops_per_launch": flops_dense,
+        },
+        "kernels": {
+            "prologue": {"ms": round(kern_ms["prologue"], 4), "GB/s": round(pro_gbs, 1),
+                         "frac_hbm": round(pro_gbs / pk["hbm_gbs"], 4),
+                         "frac_8TBs": round(pro_gbs / 8000.0, 4),
+                         "traffic": traffic.get("prologue", {}).get("bytes_per_launch")},
+            "router": {"ms": round(kern_ms["router"], 4), "pool_read_GB/s": round(router_gbs, 1)},
+            "attention_sparse": {"ms": round(kern_ms["attention_sparse"], 3), "TFLOP/s": round(sparse_tflops, 2),
+                                 "effective_dense_equiv_TFLOP/s":
+                                     round(flops_dense / (kern_ms["attention_sparse"] * 1e-3) / 1e12, 2),
+                                 "algorithmic_flops": flops_sparse},
+            "attention_dense": {"ms": round(kern_ms["attention_dense"], 3), "TFLOP/s": round(dense_tflops, 2)},
+            "sparse_speedup_incl_router": round(kern_ms["attention_dense"] /
+                                                (kern_ms["attention_sparse"] + kern_ms["router"]), 3),
+        },
+        "gpu_launches": args.steps * 5,
+        "clocks": clocks,
+        "e2e": e2e,
+    }
+    if args.cpu_baseline and world == 1:
+        line["cpu_baseline"] = cpu_baseline(d, w, args.cpu_rows)
+    return line
+
+
+# ----------------------------------------------------------------- oracle (CPU)
+
+def _oracle_inputs(d, w, sparsity):
+    import oracle
+
+    oracle.build()
+    qb = oracle.qk_norm_rope_bf16(d["q"], d["gamma_q"].numpy(), w.grid)
+    kb = oracle.qk_norm_rope_bf16(d["k"], d["gamma_k"].numpy(), w.grid)
+    idx, _ = oracle.route(qb, kb, sparsity)
+    return qb, kb, idx
+
+
+def _oracle_sample(d, w, qb, kb, idx, rows):
+    """Dense and sparse oracle attention on `rows`; returns (seconds, algorithmic FLOPs)."""
+    import oracle
+
+    N = w.N
+    t0 = time.perf_counter()
+    oracle.attention_rows(qb, kb, d["v"], rows)
+    oracle.attention_rows(qb, kb, d["v"], rows, idx)
+    dt = time.perf_counter() - t0
+    nblk = (N + 127) // 128
+    lens = np.full(nblk, 128.0)
+    lens[-1] = N - (nblk - 1) * 128
+    bh, n = rows // N, rows % N
+    sparse_keys = lens[idx.reshape(-1, nblk, idx.shape[-1])[bh, n // 128]].sum(axis=-1).sum()
+    flops = 4.0 * 96 * (len(rows) * N + sparse_keys)
+    return dt, flops
+
+
+def cpu_baseline(d, w, nrows):
+    import oracle
+    from rope_block_sparse_b200 import synth
+
+    qb, kb, idx = _oracle_inputs(d, w, SPARSITY)
+    rows = synth.sample_rows(w.B, w.heads, w.N, nrows, seed=4321).numpy()
+    dt, flops = _oracle_sample(d, w, qb, kb, idx, rows)
+    return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": oracle.threads(), "kind": "oracle",
+            "sample": f"fp64 oracle dense + sparse (0.75) attention for {len(rows)} sampled query rows of "
+                      f"{WORKLOAD} (prologue and router outputs computed by the oracle beforehand, untimed); "
+                      f"{dt:.1f} s"}
+
+
+def run_reference(args, rank, world):
+    """Reference arm: the fp64 oracle on the host cores, each step a bounded sample."""
+    if rank != 0:
+        return None
+    import oracle
+    from rope_block_sparse_b200 import synth
+
+    w = synth.WORKLOADS[WORKLOAD]
+    d = synth.draw_workload(WORKLOAD, seed=0)
+    qb, kb, idx = _oracle_inputs(d, w, SPARSITY)
+    rows_per_step = args.ref_rows
+    times, flops = [], []
+    for i in range(args.warmup + args.steps):
+        rows = synth.sample_rows(w.B, w.heads, w.N, rows_per_step, seed=1000 + i).numpy()
+        dt, fl = _oracle_sample(d, w, qb, kb, idx, rows)
+        if i >= args.warmup:
+            times.append(dt)
+            flops.append(fl)
+    value = sum(flops) / sum(times) / 1e12
+    sample = (f"fp64 oracle dense + sparse (0.75) attention for {rows_per_step} sampled query rows per step of "
+              f"{WORKLOAD}; prologue and router outputs precomputed by the oracle")
+    return {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": round(value, 6),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(1e3 * sum(times) / len(times), 3),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": f"{WORKLOAD}: B=1, 56 heads x 96, grid 31x48x84 = 124,992 tokens",
+                   "tokens": w.N, "heads": w.heads, "sparsity": SPARSITY},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": oracle.threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--workload", default=WORKLOAD, help="synthetic workload (clip32k: small profiler case)")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
+    ap.add_argument("--cpu-rows", type=int, default=1024, help="query rows of the CPU-baseline sample")
+    ap.add_argument("--ref-rows", type=int, default=128, help="query rows per reference-arm step")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+    rank, world, local = dist_setup(args.gpus)
+    try:
+        line = run_gpu(args, rank, world, local)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

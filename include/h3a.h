@@ -1,0 +1,163 @@
+/*
+ * h3a.h -- C ABI of the B200 (sm_100a) attention core for H3-style video DiTs.
+ *
+ * One DiT self-attention core per call sequence:
+ *   h3a_qk_norm_rope  fused QK-RMSNorm + 3D RoPE over Q and K
+ *   h3a_route         blockwise KV-block router (pool -> fp32 scores -> top-k)
+ *   h3a_attention     bidirectional attention, dense or over routed KV blocks
+ *
+ * Conventions shared by every call
+ *   - Tensors are bf16 (raw 16-bit words), laid out [B, N, heads, head_dim]
+ *     with head_dim contiguous and element strides given by h3a_qkv_desc.
+ *     Token n of the (T, H, W) grid is n = (t*H + h)*W + w.
+ *   - head_dim must be 96 (hidden 5376 / 56 heads), block must be 128.
+ *   - All pointers are DEVICE pointers owned by the caller, 16-byte aligned;
+ *     strides are multiples of 8 elements (16 bytes).  The library never
+ *     allocates or frees device memory; the router's scratch is a caller
+ *     workspace sized by h3a_route_workspace_size.
+ *   - Calls are asynchronous on the caller's stream.  A status other than
+ *     H3A_OK means nothing was launched, except H3A_ERR_CUDA, returned when a
+ *     launch itself failed.  Device-side failures (a bounded pipeline wait that
+ *     expired) are latched in a per-device status word and reported by
+ *     h3a_last_device_error.
+ *   - Thread safety: calls may be issued from several host threads; a call
+ *     touches only its arguments and read-only per-process state.
+ */
+#ifndef H3A_H_
+#define H3A_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* h3a_stream_t; /* a cudaStream_t; NULL = legacy default stream */
+
+typedef enum {
+    H3A_OK = 0,
+    H3A_ERR_INVALID_ARG = 1, /* null/misaligned pointer, inconsistent sizes, bad sparsity */
+    H3A_ERR_UNSUPPORTED = 2, /* head_dim != 96, block != 128, sizes beyond the int32 index range */
+    H3A_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed (see h3a_last_cuda_error_string) */
+    H3A_ERR_TIMEOUT = 4,     /* a bounded device-side wait expired; results are undefined */
+    H3A_ERR_WORKSPACE = 5    /* router workspace null or too small */
+} h3a_status;
+
+/* Token grid of one clip latent: N = T*H*W tokens. */
+typedef struct {
+    int32_t T, H, W;
+} h3a_grid;
+
+/* Shape and element strides of a [B, N, heads, head_dim] bf16 tensor.
+ * Q, K, V and O of one call share this descriptor. */
+typedef struct {
+    int32_t B, N, heads, head_dim;
+    int64_t stride_b, stride_n, stride_h; /* in elements; head_dim is contiguous */
+} h3a_qkv_desc;
+
+/* Fused QK-RMSNorm + 3D RoPE.
+ * Source: news.cocoloop.cn MiniMax-H3 SGLang report, section "Erst drei
+ * übereinandergelegte Beschleunigungsebenen" (QK-RMSNorm with 3D RoPE fused
+ * into one kernel, result unchanged); 3D multimodal RoPE and the 96-wide heads
+ * from the 52hbtv.com H3-Image page, section 二, model table.
+ * For every token n and head h of Q (and of K):
+ *   y = x / sqrt(mean(x^2) + eps) * gamma        (over the head's 96 channels)
+ *   then channels [0,32) turn with t, [32,64) with h, [64,96) with w: the pair
+ *   (32a+2j, 32a+2j+1) rotates by pos_a * theta^(-2j/32), j = 0..15;
+ *   computed in fp32, rounded once to bf16 (round to nearest even).
+ * q, k      : input tensors (device, bf16, layout d).
+ * gamma_q/k : fp32 [96] gains (device).
+ * q_out/k_out: outputs (device, layout d); may equal q/k (in place), must not
+ *             otherwise overlap them.
+ * Errors: INVALID_ARG if any pointer is null or misaligned, T*H*W != N, or
+ * eps < 0; UNSUPPORTED if head_dim != 96. */
+h3a_status h3a_qk_norm_rope(const void* q, const void* k, const h3a_qkv_desc* d,
+                            const float* gamma_q, const float* gamma_k, h3a_grid grid,
+                            double theta, float eps, void* q_out, void* k_out,
+                            h3a_stream_t stream);
+
+/* Number of KV blocks kept per query block for a given sparsity:
+ * k = clamp(ceil((1 - sparsity) * nkv - 1e-9), 1, nkv).
+ * Returns -1 if sparsity is outside [0, 1) or nkv < 1. */
+int64_t h3a_route_k(int64_t nkv, double sparsity);
+
+/* Bytes of device workspace h3a_route needs: two fp32 [B, heads, nblk, 96]
+ * pooled tensors, nblk = ceil(N / block).  Returns INVALID_ARG/UNSUPPORTED
+ * for bad descriptors. */
+h3a_status h3a_route_workspace_size(const h3a_qkv_desc* d, int32_t block, size_t* bytes);
+
+/* Blockwise KV-block router.
+ * Source: news.cocoloop.cn MiniMax-H3 SGLang report, SubBlock paragraph of
+ * section "Erst drei übereinandergelegte Beschleunigungsebenen" (a blockwise
+ * sparse router prunes the KV blocks, sparsity 0.75 or 0.80); pooling,
+ * scoring and selection as fixed by the problem statement:
+ *   qbar_i, kbar_j = fp32 means of the 128-token blocks (the tail block over
+ *   its real length), score S_ij = (qbar_i . kbar_j) / sqrt(96) in fp32,
+ *   per (b, h, i) keep the k highest scores, ties to the lower j.
+ * q, k       : prologue outputs (device, bf16, layout d).
+ * block_idx  : device int32 [B, heads, nblk, k], each row ascending.
+ * k_out      : host; receives k (may be NULL).
+ * workspace  : device, at least h3a_route_workspace_size bytes, 16-B aligned.
+ * Errors: INVALID_ARG for null pointers or sparsity outside [0, 1);
+ * UNSUPPORTED for block != 128 or head_dim != 96; WORKSPACE if the
+ * workspace is null or ws_bytes is too small. */
+h3a_status h3a_route(const void* q, const void* k, const h3a_qkv_desc* d, double sparsity,
+                     int32_t block, int32_t* block_idx, int64_t* k_out, void* workspace,
+                     size_t ws_bytes, h3a_stream_t stream);
+
+/* Bidirectional attention O = softmax(scale * Q K^T) V per (b, head).
+ * Source: dense lossless path of the news.cocoloop.cn MiniMax-H3 SGLang
+ * report (opening quote: no approximation; SSIM 1.0000) and its SubBlock
+ * sparse attention (same page; "Ein paar Grenzen": long non-causal
+ * attention, BF16).
+ * block_idx == NULL: dense, every query attends to all N keys.
+ * block_idx != NULL: device int32 [B, heads, nblk, k_blocks] routed lists
+ *   (ascending, distinct, in [0, nblk)); the queries of block i attend exactly
+ *   to the tokens of the KV blocks listed for (b, h, i), softmax renormalised
+ *   over them.
+ * scale: logit scale; 0 selects 1/sqrt(head_dim).
+ * o: output (device, bf16, layout d), must not overlap q, k or v.
+ * Tensor-core path: TMA tiles, tcgen05.mma with TMEM accumulators, fp32
+ * online softmax, one rounding of O to bf16.
+ * Errors: INVALID_ARG for null/misaligned pointers or k_blocks outside
+ * [1, nblk] in sparse mode; UNSUPPORTED for head_dim != 96, block != 128, or
+ * N >= 2^31. */
+h3a_status h3a_attention(const void* q, const void* k, const void* v, const h3a_qkv_desc* d,
+                         const int32_t* block_idx, int32_t k_blocks, int32_t block, float scale,
+                         void* o, h3a_stream_t stream);
+
+/* Human-readable name of a status. Never NULL. */
+const char* h3a_status_string(h3a_status s);
+
+/* Text of the last CUDA error seen by the calling host thread ("" if none). */
+const char* h3a_last_cuda_error_string(void);
+
+/* Synchronises `stream`, then reads and clears the current device's status
+ * word: H3A_OK, or H3A_ERR_TIMEOUT if a bounded device wait expired since the
+ * last read.  H3A_ERR_CUDA if the synchronisation itself failed. */
+h3a_status h3a_last_device_error(h3a_stream_t stream);
+
+/* Self-check of the bounded-wait path (no counterpart on the pages): launches
+ * one CTA that waits on a barrier nothing ever completes, with a limit of
+ * `limit_us` microseconds, then synchronises.  Returns H3A_ERR_TIMEOUT when
+ * the limit expired and was reported through the status word (the expected
+ * result), H3A_OK if it was not, H3A_ERR_CUDA on a CUDA failure.  Clears the
+ * status word afterwards. */
+h3a_status h3a_selftest_wait_timeout(uint32_t limit_us, h3a_stream_t stream);
+
+/* Self-check of the tensor-core building blocks used by h3a_attention (no
+ * counterpart on the pages): one CTA loads a 128x96 tile A and a 128x96 tile
+ * B (bf16, row-major, device) with TMA, computes S = A B^T (fp32 [128,128])
+ * with tcgen05.mma into tensor memory, rounds S to bf16 into tensor memory and
+ * computes R = bf16(S) C (fp32 [128,96]) with C = B read as a [128 kv, 96]
+ * MN-major operand.  Writes S and R (device fp32).  For diagnosing a new
+ * toolkit or driver. */
+h3a_status h3a_selftest_mma(const void* a, const void* b, float* s_out, float* r_out,
+                            h3a_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* H3A_H_ */

@@ -48,6 +48,12 @@ def _load():
         lib.oracle_token_position.argtypes = [i64, i32, i32, i32, P]
         lib.oracle_qk_norm_rope.argtypes = [P, i32, i64, i32, i32, P, i32, i32, i32, f64, f64, P, i32]
         lib.oracle_qk_norm_rope.restype = i32
+        lib.oracle_qk_norm_rope_tokens.argtypes = [P, i32, i64, i32, i32, P, i32, i32, i32, f64, f64, P, i64, P,
+                                                   i32]
+        lib.oracle_qk_norm_rope_tokens.restype = i32
+        lib.oracle_round_bf16.argtypes = [P, i64, P]
+        lib.oracle_qk_norm_rope_bf16.argtypes = [P, i32, i64, i32, i32, P, i32, i32, i32, f64, f64, P, i32]
+        lib.oracle_qk_norm_rope_bf16.restype = i32
         lib.oracle_num_blocks.argtypes = [i64, i32]
         lib.oracle_num_blocks.restype = i64
         lib.oracle_k_blocks.argtypes = [i64, f64]
@@ -125,6 +131,43 @@ def qk_norm_rope(x, gamma: np.ndarray, grid, theta: float = 10000.0, eps: float 
                                      theta, eps, _ptr(out), nthreads)
     if rc != 0:
         raise ValueError("oracle_qk_norm_rope: bad sizes")
+    return out
+
+
+def qk_norm_rope_tokens(x, gamma: np.ndarray, grid, tokens, theta: float = 10000.0, eps: float = 1e-6,
+                        nthreads: int = 0) -> np.ndarray:
+    """The fused prologue at flattened tokens tok = b*N + n only -> fp64 [len(tokens), heads, d]."""
+    xb = _bits(x)
+    B, N, heads, d = xb.shape
+    g = np.ascontiguousarray(gamma, dtype=np.float32)
+    tok = np.ascontiguousarray(tokens, dtype=np.int64)
+    out = np.empty((tok.size, heads, d), dtype=np.float64)
+    rc = _load().oracle_qk_norm_rope_tokens(_ptr(xb), B, N, heads, d, _ptr(g), grid[0], grid[1], grid[2], theta,
+                                            eps, _ptr(tok), tok.size, _ptr(out), nthreads)
+    if rc != 0:
+        raise ValueError("oracle_qk_norm_rope_tokens: bad sizes")
+    return out
+
+
+def round_bf16(x: np.ndarray) -> np.ndarray:
+    """Round fp64 values to bf16 (nearest-even, straight from fp64); returns uint16 bit patterns."""
+    xa = np.ascontiguousarray(x, dtype=np.float64)
+    out = np.empty(xa.shape, dtype=np.uint16)
+    _load().oracle_round_bf16(_ptr(xa), xa.size, _ptr(out))
+    return out
+
+
+def qk_norm_rope_bf16(x, gamma: np.ndarray, grid, theta: float = 10000.0, eps: float = 1e-6,
+                      nthreads: int = 0) -> np.ndarray:
+    """The fused prologue with its one rounding to bf16 applied -> uint16 bits, layout of x."""
+    xb = _bits(x)
+    B, N, heads, d = xb.shape
+    g = np.ascontiguousarray(gamma, dtype=np.float32)
+    out = np.empty(xb.shape, dtype=np.uint16)
+    rc = _load().oracle_qk_norm_rope_bf16(_ptr(xb), B, N, heads, d, _ptr(g), grid[0], grid[1], grid[2], theta,
+                                          eps, _ptr(out), nthreads)
+    if rc != 0:
+        raise ValueError("oracle_qk_norm_rope_bf16: bad sizes")
     return out
 
 

@@ -25,6 +25,7 @@
 // are listed in the repository's design notes.
 
 #include <algorithm>
+#include <cfenv>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -38,6 +39,28 @@ double bf16_to_double(uint16_t bits) {
     float f;
     std::memcpy(&f, &u, sizeof(f));
     return static_cast<double>(f);
+}
+
+// Round a double to the nearest bf16 (8 significant bits, fp32 exponent
+// range), ties to even, directly from double (no intermediate fp32 rounding).
+uint16_t double_to_bf16_rne(double x) {
+    if (std::isnan(x)) return 0x7FC0;
+    double r;
+    const double ax = std::fabs(x);
+    if (ax == 0.0) {
+        r = x;
+    } else if (ax < std::ldexp(1.0, -126)) {  // subnormal range: fixed step 2^-133
+        r = std::nearbyint(std::ldexp(x, 133)) * std::ldexp(1.0, -133);
+    } else {
+        int e;
+        std::frexp(ax, &e);  // ax in [2^(e-1), 2^e)
+        r = std::nearbyint(std::ldexp(x, 8 - e)) * std::ldexp(1.0, e - 8);
+    }
+    if (std::fabs(r) > 3.3895313892515355e38) r = std::copysign(INFINITY, x);  // beyond bf16 max
+    float f = static_cast<float>(r);  // exact: r has at most 8 significant bits
+    uint32_t u;
+    std::memcpy(&u, &f, sizeof(u));
+    return static_cast<uint16_t>(u >> 16);
 }
 
 int pick_threads(int nthreads) {
@@ -140,6 +163,60 @@ int oracle_qk_norm_rope(const uint16_t* x, int B, int64_t N, int heads, int d,
             oracle_rmsnorm(xv.data(), d, g.data(), eps, yv.data());
             oracle_rope3d(yv.data(), d, pos, theta);
             for (int c = 0; c < d; ++c) out[bshd_index(b, n, h, c, N, heads, d)] = yv[c];
+        }
+    });
+    return 0;
+}
+
+// Same as oracle_qk_norm_rope for a list of flattened tokens tok[i] = b*N + n
+// only; out layout [ntok, heads, d], fp64.
+int oracle_qk_norm_rope_tokens(const uint16_t* x, int B, int64_t N, int heads, int d, const float* gamma,
+                               int T, int H, int W, double theta, double eps, const int64_t* tok,
+                               int64_t ntok, double* out, int nthreads) {
+    if (B < 0 || N < 0 || heads <= 0 || d <= 0 || d % 6 != 0) return -1;
+    if (static_cast<int64_t>(T) * H * W != N) return -1;
+    std::vector<double> g(d);
+    for (int i = 0; i < d; ++i) g[i] = static_cast<double>(gamma[i]);
+    parallel_for(ntok, nthreads, [&](int64_t i) {
+        int b = static_cast<int>(tok[i] / N);
+        int64_t n = tok[i] % N;
+        int pos[3];
+        oracle_token_position(n, T, H, W, pos);
+        std::vector<double> xv(d), yv(d);
+        for (int h = 0; h < heads; ++h) {
+            for (int c = 0; c < d; ++c) xv[c] = bf16_to_double(x[bshd_index(b, n, h, c, N, heads, d)]);
+            oracle_rmsnorm(xv.data(), d, g.data(), eps, yv.data());
+            oracle_rope3d(yv.data(), d, pos, theta);
+            for (int c = 0; c < d; ++c) out[(i * heads + h) * d + c] = yv[c];
+        }
+    });
+    return 0;
+}
+
+// Round doubles to bf16 bit patterns, nearest-even.
+void oracle_round_bf16(const double* x, int64_t n, uint16_t* out) {
+    for (int64_t i = 0; i < n; ++i) out[i] = double_to_bf16_rne(x[i]);
+}
+
+// The fused prologue with its single rounding to bf16 applied, for whole
+// tensors too large to hold in fp64: out is bf16 bits, layout of x.
+int oracle_qk_norm_rope_bf16(const uint16_t* x, int B, int64_t N, int heads, int d, const float* gamma,
+                             int T, int H, int W, double theta, double eps, uint16_t* out, int nthreads) {
+    if (B < 0 || N < 0 || heads <= 0 || d <= 0 || d % 6 != 0) return -1;
+    if (static_cast<int64_t>(T) * H * W != N) return -1;
+    std::vector<double> g(d);
+    for (int i = 0; i < d; ++i) g[i] = static_cast<double>(gamma[i]);
+    parallel_for(static_cast<int64_t>(B) * N, nthreads, [&](int64_t bn) {
+        int b = static_cast<int>(bn / N);
+        int64_t n = bn % N;
+        int pos[3];
+        oracle_token_position(n, T, H, W, pos);
+        std::vector<double> xv(d), yv(d);
+        for (int h = 0; h < heads; ++h) {
+            for (int c = 0; c < d; ++c) xv[c] = bf16_to_double(x[bshd_index(b, n, h, c, N, heads, d)]);
+            oracle_rmsnorm(xv.data(), d, g.data(), eps, yv.data());
+            oracle_rope3d(yv.data(), d, pos, theta);
+            for (int c = 0; c < d; ++c) out[bshd_index(b, n, h, c, N, heads, d)] = double_to_bf16_rne(yv[c]);
         }
     });
     return 0;

@@ -1,1 +1,16 @@
-"""B200-native attention core for H3-style video DiTs."""
+"""B200-native (sm_100a) attention core for H3-style video DiTs.
+
+Public API (CUDA tensors, bf16 [B, N, heads, 96]):
+    qk_norm_rope(q, k, gamma_q, gamma_k, grid, theta, eps) -> (q', k')
+    route(q, k, sparsity) -> int32 [B, heads, nblk, k] KV-block lists
+    attention(q, k, v, block_idx=None) -> o
+    attention_core(q, k, v, gamma_q, gamma_k, grid, sparsity=None) -> (o, block_idx)
+
+All compute runs in libh3a.so (include/h3a.h); the Python layer only marshals
+arguments.  ``synth`` holds the seeded synthetic input generators.
+"""
+from .h3a import (H3AError, attention, attention_core, last_device_error, load, qk_norm_rope, route,
+                  route_k, route_workspace_size, selftest_mma, selftest_wait_timeout)
+
+__all__ = ["H3AError", "attention", "attention_core", "last_device_error", "load", "qk_norm_rope", "route",
+           "route_k", "route_workspace_size", "selftest_mma", "selftest_wait_timeout"]

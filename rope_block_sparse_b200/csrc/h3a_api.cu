@@ -1,0 +1,264 @@
+// C-ABI front end of libh3a: argument validation, tensor-map encoding and
+// launches on the caller's stream.  Nothing here allocates device memory; the
+// only device state is the per-device status word below.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "h3a.h"
+#include "h3a_internal.h"
+
+// Sticky per-device status word: kernels OR error bits into it.
+__device__ int g_h3a_status_word;
+
+namespace h3a {
+namespace {
+
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per pipeline wait
+constexpr int kMaxDevices = 64;
+
+thread_local std::string g_last_cuda_error;
+
+h3a_status cuda_fail(cudaError_t e) {
+    g_last_cuda_error = std::string(cudaGetErrorName(e)) + ": " + cudaGetErrorString(e);
+    return H3A_ERR_CUDA;
+}
+
+// Device address of g_h3a_status_word, resolved once per device.
+std::mutex g_status_mu;
+int* g_status_ptr[kMaxDevices] = {};
+
+h3a_status status_word(int** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (dev < 0 || dev >= kMaxDevices) return H3A_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_status_mu);
+    if (g_status_ptr[dev] == nullptr) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_h3a_status_word);
+        if (e != cudaSuccess) return cuda_fail(e);
+        g_status_ptr[dev] = static_cast<int*>(p);
+    }
+    *out = g_status_ptr[dev];
+    return H3A_OK;
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+std::once_flag g_encode_once;
+EncodeTiledFn g_encode = nullptr;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Validates a Q/K/V/O descriptor.  Fills `s` on success.
+h3a_status check_desc(const h3a_qkv_desc* d, Shape* s) {
+    if (d == nullptr) return H3A_ERR_INVALID_ARG;
+    if (d->head_dim != kHeadDim) return H3A_ERR_UNSUPPORTED;
+    if (d->B < 1 || d->N < 1 || d->heads < 1) return H3A_ERR_INVALID_ARG;
+    if (d->stride_b < 0 || d->stride_n < 0 || d->stride_h < 0) return H3A_ERR_INVALID_ARG;
+    if ((d->stride_b % 8) || (d->stride_n % 8) || (d->stride_h % 8)) return H3A_ERR_INVALID_ARG;
+    if (d->heads > 1 && d->stride_h < kHeadDim) return H3A_ERR_INVALID_ARG;
+    if (d->N > 1 && d->stride_n < kHeadDim) return H3A_ERR_INVALID_ARG;
+    // byte strides must stay within the tensor-map limit (2^40)
+    const int64_t lim = (int64_t(1) << 39);
+    if (d->stride_b >= lim || d->stride_n >= lim || d->stride_h >= lim) return H3A_ERR_UNSUPPORTED;
+    s->B = d->B;
+    s->N = d->N;
+    s->heads = d->heads;
+    s->sb = d->stride_b;
+    s->sn = d->stride_n;
+    s->sh = d->stride_h;
+    return H3A_OK;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+size_t pooled_bytes(const Shape& s, int nblk) {
+    return align256(static_cast<size_t>(s.B) * s.heads * nblk * kHeadDim * sizeof(float));
+}
+
+}  // namespace
+
+cudaError_t make_qkv_tensor_map(CUtensorMap* map, const void* base, const Shape& s) {
+    std::call_once(g_encode_once, []() {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    });
+    if (g_encode == nullptr) return cudaErrorNotSupported;
+    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(kHeadDim), static_cast<cuuint64_t>(s.heads),
+                                static_cast<cuuint64_t>(s.N), static_cast<cuuint64_t>(s.B)};
+    // byte strides of dims 1..3; a size-1 dim gets a nominal (unused) stride
+    auto stride_or = [](int64_t st, int64_t fallback) { return static_cast<cuuint64_t>((st > 0 ? st : fallback) * 2); };
+    const cuuint64_t strides[3] = {stride_or(s.sh, kHeadDim), stride_or(s.sn, kHeadDim),
+                                   stride_or(s.sb, kHeadDim)};
+    const cuuint32_t box[4] = {32, 1, 128, 1};
+    const cuuint32_t elem_strides[4] = {1, 1, 1, 1};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
+                          elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+}  // namespace h3a
+
+using namespace h3a;
+
+extern "C" {
+
+const char* h3a_status_string(h3a_status s) {
+    switch (s) {
+        case H3A_OK: return "H3A_OK";
+        case H3A_ERR_INVALID_ARG: return "H3A_ERR_INVALID_ARG";
+        case H3A_ERR_UNSUPPORTED: return "H3A_ERR_UNSUPPORTED";
+        case H3A_ERR_CUDA: return "H3A_ERR_CUDA";
+        case H3A_ERR_TIMEOUT: return "H3A_ERR_TIMEOUT";
+        case H3A_ERR_WORKSPACE: return "H3A_ERR_WORKSPACE";
+    }
+    return "H3A_ERR_UNKNOWN";
+}
+
+const char* h3a_last_cuda_error_string(void) { return g_last_cuda_error.c_str(); }
+
+h3a_status h3a_qk_norm_rope(const void* q, const void* k, const h3a_qkv_desc* d, const float* gamma_q,
+                            const float* gamma_k, h3a_grid grid, double theta, float eps, void* q_out, void* k_out,
+                            h3a_stream_t stream) {
+    Shape s;
+    h3a_status rc = check_desc(d, &s);
+    if (rc != H3A_OK) return rc;
+    if (!q || !k || !gamma_q || !gamma_k || !q_out || !k_out) return H3A_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(q_out) || !aligned16(k_out)) return H3A_ERR_INVALID_ARG;
+    if (!(reinterpret_cast<uintptr_t>(gamma_q) % 4 == 0 && reinterpret_cast<uintptr_t>(gamma_k) % 4 == 0))
+        return H3A_ERR_INVALID_ARG;
+    if (grid.T < 1 || grid.H < 1 || grid.W < 1) return H3A_ERR_INVALID_ARG;
+    if (static_cast<int64_t>(grid.T) * grid.H * grid.W != d->N) return H3A_ERR_INVALID_ARG;
+    if (!(eps >= 0.0f) || !(theta > 0.0)) return H3A_ERR_INVALID_ARG;
+    cudaError_t e = launch_qk_norm_rope(q, k, q_out, k_out, gamma_q, gamma_k, s, grid.T, grid.H, grid.W, theta, eps,
+                                        reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? H3A_OK : cuda_fail(e);
+}
+
+int64_t h3a_route_k(int64_t nkv, double sparsity) {
+    if (nkv < 1 || !(sparsity >= 0.0 && sparsity < 1.0)) return -1;
+    int64_t kk = static_cast<int64_t>(std::ceil((1.0 - sparsity) * static_cast<double>(nkv) - 1e-9));
+    if (kk < 1) kk = 1;
+    if (kk > nkv) kk = nkv;
+    return kk;
+}
+
+h3a_status h3a_route_workspace_size(const h3a_qkv_desc* d, int32_t block, size_t* bytes) {
+    Shape s;
+    h3a_status rc = check_desc(d, &s);
+    if (rc != H3A_OK) return rc;
+    if (bytes == nullptr) return H3A_ERR_INVALID_ARG;
+    if (block != kBlock) return H3A_ERR_UNSUPPORTED;
+    const int nblk = (s.N + kBlock - 1) / kBlock;
+    *bytes = 2 * pooled_bytes(s, nblk);
+    return H3A_OK;
+}
+
+h3a_status h3a_route(const void* q, const void* k, const h3a_qkv_desc* d, double sparsity, int32_t block,
+                     int32_t* block_idx, int64_t* k_out, void* workspace, size_t ws_bytes, h3a_stream_t stream) {
+    Shape s;
+    h3a_status rc = check_desc(d, &s);
+    if (rc != H3A_OK) return rc;
+    if (block != kBlock) return H3A_ERR_UNSUPPORTED;
+    if (!q || !k || !block_idx) return H3A_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || (reinterpret_cast<uintptr_t>(block_idx) & 3u)) return H3A_ERR_INVALID_ARG;
+    if (!(sparsity >= 0.0 && sparsity < 1.0)) return H3A_ERR_INVALID_ARG;
+    const int nblk = (s.N + kBlock - 1) / kBlock;
+    if (nblk > route_max_blocks()) return H3A_ERR_UNSUPPORTED;
+    if (static_cast<int64_t>(s.B) * s.heads > 65535) return H3A_ERR_UNSUPPORTED;
+    const size_t half = pooled_bytes(s, nblk);
+    if (workspace == nullptr || !aligned16(workspace) || ws_bytes < 2 * half) return H3A_ERR_WORKSPACE;
+    const int64_t kk = h3a_route_k(nblk, sparsity);
+    if (k_out) *k_out = kk;
+    float* pq = static_cast<float*>(workspace);
+    float* pk = reinterpret_cast<float*>(static_cast<char*>(workspace) + half);
+    cudaError_t e = launch_route(q, k, s, nblk, static_cast<int>(kk), pq, pk, block_idx,
+                                 reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? H3A_OK : cuda_fail(e);
+}
+
+h3a_status h3a_attention(const void* q, const void* k, const void* v, const h3a_qkv_desc* d,
+                         const int32_t* block_idx, int32_t k_blocks, int32_t block, float scale, void* o,
+                         h3a_stream_t stream) {
+    Shape s;
+    h3a_status rc = check_desc(d, &s);
+    if (rc != H3A_OK) return rc;
+    if (block != kBlock) return H3A_ERR_UNSUPPORTED;
+    if (!q || !k || !v || !o) return H3A_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return H3A_ERR_INVALID_ARG;
+    if (!(scale >= 0.0f) || !std::isfinite(scale)) return H3A_ERR_INVALID_ARG;
+    const int nblk = (s.N + kBlock - 1) / kBlock;
+    if (block_idx != nullptr) {
+        if ((reinterpret_cast<uintptr_t>(block_idx) & 3u) || k_blocks < 1 || k_blocks > nblk)
+            return H3A_ERR_INVALID_ARG;
+    }
+    const int64_t grid = static_cast<int64_t>(s.B) * s.heads * ((nblk + 1) / 2);
+    if (grid >= (int64_t(1) << 31)) return H3A_ERR_UNSUPPORTED;
+    if (scale == 0.0f) scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(kHeadDim)));
+    int* status = nullptr;
+    rc = status_word(&status);
+    if (rc != H3A_OK) return rc;
+    CUtensorMap tq, tk, tv;
+    cudaError_t e = make_qkv_tensor_map(&tq, q, s);
+    if (e == cudaSuccess) e = make_qkv_tensor_map(&tk, k, s);
+    if (e == cudaSuccess) e = make_qkv_tensor_map(&tv, v, s);
+    if (e != cudaSuccess) return cuda_fail(e);
+    e = launch_attention(tq, tk, tv, o, s, block_idx, k_blocks, scale, status, kWaitLimitNs,
+                         reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? H3A_OK : cuda_fail(e);
+}
+
+h3a_status h3a_last_device_error(h3a_stream_t stream) {
+    int* status = nullptr;
+    h3a_status rc = status_word(&status);
+    if (rc != H3A_OK) return rc;
+    cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e);
+    int word = 0;
+    const int zero = 0;
+    e = cudaMemcpyFromSymbol(&word, g_h3a_status_word, sizeof(int));
+    if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_h3a_status_word, &zero, sizeof(int));
+    if (e != cudaSuccess) return cuda_fail(e);
+    return (word & kDevTimeout) ? H3A_ERR_TIMEOUT : H3A_OK;
+}
+
+h3a_status h3a_selftest_wait_timeout(uint32_t limit_us, h3a_stream_t stream) {
+    int* status = nullptr;
+    h3a_status rc = status_word(&status);
+    if (rc != H3A_OK) return rc;
+    rc = h3a_last_device_error(stream);  // start from a clear word
+    if (rc == H3A_ERR_CUDA) return rc;
+    cudaError_t e = launch_selftest_wait(static_cast<uint64_t>(limit_us) * 1000ull, status,
+                                         reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e);
+    return h3a_last_device_error(stream);
+}
+
+h3a_status h3a_selftest_mma(const void* a, const void* b, float* s_out, float* r_out, h3a_stream_t stream) {
+    if (!a || !b || !s_out || !r_out) return H3A_ERR_INVALID_ARG;
+    if (!aligned16(a) || !aligned16(b) || !aligned16(s_out) || !aligned16(r_out)) return H3A_ERR_INVALID_ARG;
+    int* status = nullptr;
+    h3a_status rc = status_word(&status);
+    if (rc != H3A_OK) return rc;
+    Shape s{1, 128, 1, 128 * kHeadDim, kHeadDim, kHeadDim};
+    CUtensorMap ta, tb;
+    cudaError_t e = make_qkv_tensor_map(&ta, a, s);
+    if (e == cudaSuccess) e = make_qkv_tensor_map(&tb, b, s);
+    if (e != cudaSuccess) return cuda_fail(e);
+    e = launch_selftest_mma(ta, tb, s_out, r_out, status, kWaitLimitNs, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? H3A_OK : cuda_fail(e);
+}
+
+}  // extern "C"

@@ -1,0 +1,48 @@
+// Launchers shared between the C-ABI front end (h3a_api.cu) and the kernel
+// translation units.  Not part of the public interface.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+namespace h3a {
+
+constexpr int kHeadDim = 96;
+constexpr int kBlock = 128;
+
+// Status word bits set by kernels (read back by h3a_last_device_error).
+constexpr int kDevTimeout = 1;
+
+struct Shape {
+    int B, N, heads;
+    int64_t sb, sn, sh;  // element strides; head_dim contiguous
+};
+
+// QK-RMSNorm + 3D RoPE (prologue.cu).
+cudaError_t launch_qk_norm_rope(const void* q, const void* k, void* q_out, void* k_out, const float* gamma_q,
+                                const float* gamma_k, const Shape& s, int T, int H, int W, double theta,
+                                float eps, cudaStream_t st);
+
+// Router (router.cu): block means of q and k into pooled_q / pooled_k
+// ([B, heads, nblk, 96] fp32), then scores and top-k into idx.
+cudaError_t launch_route(const void* q, const void* k, const Shape& s, int nblk, int kk, float* pooled_q,
+                         float* pooled_k, int32_t* idx, cudaStream_t st);
+// Largest nblk the score/top-k kernel supports (shared-memory bound).
+int route_max_blocks();
+
+// Attention (attention.cu).  blocks == nullptr: dense.
+cudaError_t launch_attention(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, void* o,
+                             const Shape& s, const int32_t* blocks, int k_blocks, float scale, int* status,
+                             uint64_t timeout_ns, cudaStream_t st);
+
+// Self-checks (selftest.cu).
+cudaError_t launch_selftest_wait(uint64_t limit_ns, int* status, cudaStream_t st);
+cudaError_t launch_selftest_mma(const CUtensorMap& ta, const CUtensorMap& tb, float* s_out, float* r_out,
+                                int* status, uint64_t timeout_ns, cudaStream_t st);
+
+// Tensor map over a [B, N, heads, 96] bf16 tensor with a {32, 1, 128, 1} box,
+// 64-byte swizzle (h3a_api.cu).
+cudaError_t make_qkv_tensor_map(CUtensorMap* map, const void* base, const Shape& s);
+
+}  // namespace h3a

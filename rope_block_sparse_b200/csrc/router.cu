@@ -1,0 +1,285 @@
+// Blockwise KV-block router (news.cocoloop.cn MiniMax-H3 SGLang report,
+// SubBlock paragraph: a blockwise sparse router prunes the KV blocks taking
+// part in attention, sparsity 0.75 or 0.80).  Pooling, scoring and selection
+// follow the problem statement: mean-pooled 128-token blocks, fp32 scores,
+// per-query-block top-k with ties to the lower block index.
+//
+// Two kernels:
+//   block_pool_kernel   HBM-bound: one CTA per (batch, block, tensor) streams the
+//                       block's 128 token rows (all heads) once and writes fp32
+//                       means [B, heads, nblk, 96].
+//   score_topk_kernel   one CTA per (batch*head, 16 query blocks): fp32 scores of
+//                       its query blocks against every key block into shared
+//                       memory, then one warp per query block selects the top k
+//                       with a 4-pass 8-bit radix select over order-preserving
+//                       32-bit keys and emits the indices in ascending order.
+#include <cuda_bf16.h>
+
+#include <cmath>
+
+#include "h3a_internal.h"
+
+namespace h3a {
+namespace {
+
+constexpr int kPoolThreads = 224;    // 672 16-byte vectors per 56-head token row, 3 per thread
+constexpr int kVecPerThread = 3;
+constexpr int kHeadsPerPoolCta = kPoolThreads * kVecPerThread / (kHeadDim / 8);  // 56
+constexpr int kScoreThreads = 512;   // 16 warps
+constexpr int kRowsPerCta = 16;      // query blocks per score CTA (one warp each)
+constexpr int kScoreSmemLimit = 200 * 1024;
+
+struct PoolArgs {
+    const __nv_bfloat16* x[2];
+    float* out[2];
+    int N, heads, nblk;
+    int64_t sb, sn, sh;
+};
+
+__device__ __forceinline__ void acc8(float* acc, uint4 v) {
+    acc[0] += __uint_as_float(v.x << 16);
+    acc[1] += __uint_as_float(v.x & 0xFFFF0000u);
+    acc[2] += __uint_as_float(v.y << 16);
+    acc[3] += __uint_as_float(v.y & 0xFFFF0000u);
+    acc[4] += __uint_as_float(v.z << 16);
+    acc[5] += __uint_as_float(v.z & 0xFFFF0000u);
+    acc[6] += __uint_as_float(v.w << 16);
+    acc[7] += __uint_as_float(v.w & 0xFFFF0000u);
+}
+
+// grid: (nblk, B, 2 tensors x head chunks of 56).  Thread t covers 16-byte
+// vectors t, t+224, t+448 of the chunk's part of a token row (vector v = head
+// 56*chunk + v/12, channels 8*(v%12) .. +7).
+__global__ void __launch_bounds__(kPoolThreads) block_pool_kernel(const PoolArgs a) {
+    const int blk = blockIdx.x, b = blockIdx.y, which = blockIdx.z & 1, chunk = blockIdx.z >> 1;
+    const __nv_bfloat16* x = a.x[which];
+    const int n0 = blk * kBlock;
+    const int n1 = min(a.N, n0 + kBlock);
+    const int h_base = chunk * kHeadsPerPoolCta;
+    const int vec_per_row = min(kHeadsPerPoolCta, a.heads - h_base) * (kHeadDim / 8);
+
+    int64_t off[kVecPerThread];
+    bool act[kVecPerThread];
+#pragma unroll
+    for (int u = 0; u < kVecPerThread; ++u) {
+        const int v = threadIdx.x + u * kPoolThreads;
+        act[u] = v < vec_per_row;
+        const int h = h_base + v / (kHeadDim / 8), c = (v % (kHeadDim / 8)) * 8;
+        off[u] = static_cast<int64_t>(b) * a.sb + static_cast<int64_t>(h) * a.sh + c;
+    }
+    float acc[kVecPerThread][8];
+#pragma unroll
+    for (int u = 0; u < kVecPerThread; ++u)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[u][i] = 0.f;
+
+    int n = n0;
+    for (; n + 4 <= n1; n += 4) {
+        uint4 v[4][kVecPerThread];
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+#pragma unroll
+            for (int u = 0; u < kVecPerThread; ++u)
+                v[r][u] = act[u] ? __ldg(reinterpret_cast<const uint4*>(x + off[u] + static_cast<int64_t>(n + r) * a.sn))
+                                 : make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+#pragma unroll
+            for (int u = 0; u < kVecPerThread; ++u) acc8(acc[u], v[r][u]);
+    }
+    for (; n < n1; ++n) {
+#pragma unroll
+        for (int u = 0; u < kVecPerThread; ++u)
+            if (act[u]) acc8(acc[u], __ldg(reinterpret_cast<const uint4*>(x + off[u] + static_cast<int64_t>(n) * a.sn)));
+    }
+    const float inv_len = 1.0f / static_cast<float>(n1 - n0);
+#pragma unroll
+    for (int u = 0; u < kVecPerThread; ++u) {
+        if (!act[u]) continue;
+        const int v = threadIdx.x + u * kPoolThreads;
+        const int h = h_base + v / (kHeadDim / 8), c = (v % (kHeadDim / 8)) * 8;
+        float* dst = a.out[which] + ((static_cast<int64_t>(b) * a.heads + h) * a.nblk + blk) * kHeadDim + c;
+        float4 lo = make_float4(acc[u][0] * inv_len, acc[u][1] * inv_len, acc[u][2] * inv_len, acc[u][3] * inv_len);
+        float4 hi = make_float4(acc[u][4] * inv_len, acc[u][5] * inv_len, acc[u][6] * inv_len, acc[u][7] * inv_len);
+        reinterpret_cast<float4*>(dst)[0] = lo;
+        reinterpret_cast<float4*>(dst)[1] = hi;
+    }
+}
+
+struct ScoreArgs {
+    const float* qp;
+    const float* kp;
+    int32_t* idx;
+    int nblk, kk;
+    float inv_sqrt_d;
+};
+
+// Order-preserving map of a finite float to uint32 (-0 folded onto +0).
+__device__ __forceinline__ uint32_t order_key(float f) {
+    uint32_t u = __float_as_uint(f == 0.f ? 0.f : f);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// grid: (ceil(nblk / 16), B*heads).  Dynamic shared memory:
+// qbar[16][96] fp32, scores[16][nblk] fp32, histograms[16][256] u32.
+__global__ void __launch_bounds__(kScoreThreads) score_topk_kernel(const ScoreArgs a) {
+    extern __shared__ __align__(16) float smem[];
+    float* qbar = smem;                                   // [16][96]
+    float* scores = qbar + kRowsPerCta * kHeadDim;        // [16][nblk]
+    uint32_t* hist = reinterpret_cast<uint32_t*>(scores + kRowsPerCta * a.nblk);  // [16][256]
+
+    const int bh = blockIdx.y;
+    const int i0 = blockIdx.x * kRowsPerCta;
+    const int rows = min(kRowsPerCta, a.nblk - i0);
+    const float* qsrc = a.qp + (static_cast<int64_t>(bh) * a.nblk + i0) * kHeadDim;
+    const float* ksrc = a.kp + static_cast<int64_t>(bh) * a.nblk * kHeadDim;
+
+    for (int e = threadIdx.x; e < kRowsPerCta * kHeadDim; e += kScoreThreads)
+        qbar[e] = (e < rows * kHeadDim) ? qsrc[e] : 0.f;
+    __syncthreads();
+
+    // scores[r][j] = (qbar_r . kbar_j) * inv_sqrt_d, dot in channel order
+    for (int j = threadIdx.x; j < a.nblk; j += kScoreThreads) {
+        float dot[kRowsPerCta];
+#pragma unroll
+        for (int r = 0; r < kRowsPerCta; ++r) dot[r] = 0.f;
+        const float4* kj = reinterpret_cast<const float4*>(ksrc + static_cast<int64_t>(j) * kHeadDim);
+#pragma unroll 4
+        for (int c4 = 0; c4 < kHeadDim / 4; ++c4) {
+            const float4 kv = __ldg(kj + c4);
+#pragma unroll
+            for (int r = 0; r < kRowsPerCta; ++r) {
+                const float4 qv = reinterpret_cast<const float4*>(qbar + r * kHeadDim)[c4];
+                dot[r] = fmaf(qv.x, kv.x, dot[r]);
+                dot[r] = fmaf(qv.y, kv.y, dot[r]);
+                dot[r] = fmaf(qv.z, kv.z, dot[r]);
+                dot[r] = fmaf(qv.w, kv.w, dot[r]);
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < kRowsPerCta; ++r) scores[r * a.nblk + j] = dot[r] * a.inv_sqrt_d;
+    }
+    __syncthreads();
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (warp >= rows) return;
+    const float* s = scores + warp * a.nblk;
+    uint32_t* h = hist + warp * 256;
+
+    // radix select of the kk-th largest key, 8 bits per pass, most significant first
+    uint32_t prefix = 0;
+    int remaining = a.kk;
+    for (int shift = 24; shift >= 0; shift -= 8) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) h[lane * 8 + i] = 0u;
+        __syncwarp();
+        const uint32_t hi_mask = (shift == 24) ? 0u : (0xFFFFFFFFu << (shift + 8));
+        for (int j = lane; j < a.nblk; j += 32) {
+            const uint32_t u = order_key(s[j]);
+            if ((u & hi_mask) == (prefix & hi_mask)) atomicAdd(&h[(u >> shift) & 255u], 1u);
+        }
+        __syncwarp();
+        // lane l owns digits 255-8l .. 248-8l (descending)
+        uint32_t cnt[8];
+        uint32_t local = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            cnt[i] = h[255 - (lane * 8 + i)];
+            local += cnt[i];
+        }
+        uint32_t incl = local;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += t;
+        }
+        const uint32_t excl = incl - local;  // keys with a larger digit, from lanes before
+        const bool mine = excl < static_cast<uint32_t>(remaining) && static_cast<uint32_t>(remaining) <= incl;
+        const uint32_t owner = __ballot_sync(0xffffffffu, mine);
+        const int src = __ffs(owner) - 1;
+        uint32_t digit = 0, above = 0;
+        if (mine) {
+            uint32_t run = excl;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                if (run < static_cast<uint32_t>(remaining) && static_cast<uint32_t>(remaining) <= run + cnt[i]) {
+                    digit = 255 - (lane * 8 + i);
+                    above = run;
+                    break;
+                }
+                run += cnt[i];
+            }
+        }
+        digit = __shfl_sync(0xffffffffu, digit, src);
+        above = __shfl_sync(0xffffffffu, above, src);
+        prefix |= digit << shift;
+        remaining -= static_cast<int>(above);
+        __syncwarp();
+    }
+
+    // emit: every key above the threshold, plus the first `remaining` keys equal
+    // to it (lowest indices first), in ascending index order
+    int32_t* out = a.idx + (static_cast<int64_t>(bh) * a.nblk + i0 + warp) * a.kk;
+    const uint32_t lt_mask = (1u << lane) - 1u;
+    int written = 0, eq_seen = 0;
+    for (int base = 0; base < a.nblk; base += 32) {
+        const int j = base + lane;
+        const bool in = j < a.nblk;
+        const uint32_t u = in ? order_key(s[j]) : 0u;
+        const bool gt = in && u > prefix;
+        const bool eq = in && u == prefix;
+        const uint32_t eq_mask = __ballot_sync(0xffffffffu, eq);
+        const int eq_rank = eq_seen + __popc(eq_mask & lt_mask);
+        const bool sel = gt || (eq && eq_rank < remaining);
+        const uint32_t sel_mask = __ballot_sync(0xffffffffu, sel);
+        if (sel) out[written + __popc(sel_mask & lt_mask)] = j;
+        written += __popc(sel_mask);
+        eq_seen += __popc(eq_mask);
+    }
+}
+
+size_t score_smem_bytes(int nblk) {
+    return (static_cast<size_t>(kRowsPerCta) * kHeadDim + static_cast<size_t>(kRowsPerCta) * nblk) * sizeof(float) +
+           static_cast<size_t>(kRowsPerCta) * 256 * sizeof(uint32_t);
+}
+
+}  // namespace
+
+int route_max_blocks() {
+    // largest nblk whose score tile fits the shared-memory budget
+    return static_cast<int>((kScoreSmemLimit - score_smem_bytes(0)) / (kRowsPerCta * sizeof(float)));
+}
+
+cudaError_t launch_route(const void* q, const void* k, const Shape& s, int nblk, int kk, float* pooled_q,
+                         float* pooled_k, int32_t* idx, cudaStream_t st) {
+    PoolArgs p;
+    p.x[0] = static_cast<const __nv_bfloat16*>(q);
+    p.x[1] = static_cast<const __nv_bfloat16*>(k);
+    p.out[0] = pooled_q;
+    p.out[1] = pooled_k;
+    p.N = s.N;
+    p.heads = s.heads;
+    p.nblk = nblk;
+    p.sb = s.sb;
+    p.sn = s.sn;
+    p.sh = s.sh;
+    const int chunks = (s.heads + kHeadsPerPoolCta - 1) / kHeadsPerPoolCta;
+    block_pool_kernel<<<dim3(nblk, s.B, 2 * chunks), kPoolThreads, 0, st>>>(p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+
+    ScoreArgs a;
+    a.qp = pooled_q;
+    a.kp = pooled_k;
+    a.idx = idx;
+    a.nblk = nblk;
+    a.kk = kk;
+    a.inv_sqrt_d = static_cast<float>(1.0 / std::sqrt(static_cast<double>(kHeadDim)));
+    const size_t smem = score_smem_bytes(nblk);
+    e = cudaFuncSetAttribute(score_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    score_topk_kernel<<<dim3((nblk + kRowsPerCta - 1) / kRowsPerCta, s.B * s.heads), kScoreThreads, smem, st>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace h3a

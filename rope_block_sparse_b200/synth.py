@@ -58,6 +58,8 @@ WORKLOADS = {
     "video5s_sparse": Workload("video5s_sparse", 1, 56, (31, 48, 84), "structured", 0.75),
     # 10 s clip latent: 61x48x84 = 245,952 tokens, block-sparse at 0.80 plus a dense run.
     "video10s": Workload("video10s", 1, 56, (61, 48, 84), "structured", 0.80, also_dense=True),
+    # a 16x32x64 = 32,768-token clip for profiler captures: Q, K, V still exceed L2 (352 MB each).
+    "clip32k": Workload("clip32k", 1, 56, (16, 32, 64), "structured", 0.75),
 }
 
 _STREAM = {"q": 1, "k": 2, "v": 3, "gamma_q": 4, "gamma_k": 5}

@@ -1,0 +1,193 @@
+"""GPU parity on sizes the oracle finishes in seconds: every output compared.
+
+Inputs of each stage come from the seeded generator or from the oracle (its
+prologue output, its block lists), never from a CUDA kernel, so each kernel is
+checked on its own; test_gpu_chain.py checks the stages run back to back.
+"""
+import numpy as np
+import pytest
+import torch
+
+import rope_block_sparse_b200 as h3a
+from rope_block_sparse_b200 import synth
+from helpers import (bits, check_attention, check_prologue, check_router, from_bits, gather_rows)
+
+pytestmark = [pytest.mark.gpu,
+              pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")]
+
+THETA, EPS = 10000.0, 1e-6
+
+
+def _inputs(B, heads, grid, dist="normal", seed=0):
+    return synth.draw(B, heads, grid, dist, seed)
+
+
+def _dev(t):
+    return t.cuda()
+
+
+# ---------------------------------------------------------------- self-checks
+
+def test_selftest_mma_matches_torch():
+    g = torch.Generator().manual_seed(3)
+    a = torch.randn(128, 96, generator=g).to(torch.bfloat16)
+    b = torch.randn(128, 96, generator=g).to(torch.bfloat16)
+    s, r = h3a.selftest_mma(a.cuda(), b.cuda())
+    torch.cuda.synchronize()
+    assert h3a.last_device_error() == 0
+    s_ref = a.double() @ b.double().T
+    assert torch.allclose(s.cpu().double(), s_ref, rtol=0, atol=2e-3)
+    r_ref = s.cpu().to(torch.bfloat16).double() @ b.double()
+    assert torch.allclose(r.cpu().double(), r_ref, rtol=0, atol=2e-2)
+
+
+def test_bounded_wait_reports_timeout_and_context_survives():
+    assert h3a.selftest_wait_timeout(2000) == 4  # H3A_ERR_TIMEOUT
+    assert h3a.last_device_error() == 0          # cleared
+    d = _inputs(1, 2, (2, 4, 8))
+    q, k, v = (_dev(d[n]) for n in "qkv")
+    o = h3a.attention(q, k, v)
+    torch.cuda.synchronize()
+    assert h3a.last_device_error() == 0 and torch.isfinite(o.float()).all()
+
+
+# ---------------------------------------------------------------- prologue
+
+PROLOGUE_CASES = [
+    ("tiny", 1, 2, (2, 4, 8), "normal"),
+    ("layer8k", 1, 56, (8, 24, 42), "head_scaled"),
+    ("ragged", 2, 5, (3, 5, 7), "normal"),
+    ("heads57", 1, 57, (2, 3, 4), "normal"),
+]
+
+
+@pytest.mark.parametrize("name,B,heads,grid,dist", PROLOGUE_CASES, ids=[c[0] for c in PROLOGUE_CASES])
+def test_prologue_parity(orc, name, B, heads, grid, dist):
+    d = _inputs(B, heads, grid, dist)
+    qo, ko = h3a.qk_norm_rope(_dev(d["q"]), _dev(d["k"]), _dev(d["gamma_q"]), _dev(d["gamma_k"]), grid, THETA, EPS)
+    torch.cuda.synchronize()
+    for x, g, out in ((d["q"], d["gamma_q"], qo), (d["k"], d["gamma_k"], ko)):
+        want = orc.qk_norm_rope_bf16(x, g.numpy(), grid, THETA, EPS)
+        check_prologue(bits(out), want, name)
+
+
+def test_prologue_strided_and_inplace(orc):
+    """Heads 0..4 of a 7-head buffer (token stride 7*96), in place."""
+    grid, heads = (2, 6, 5), 5
+    d = _inputs(1, 7, grid)
+    qbuf, kbuf = _dev(d["q"]), _dev(d["k"])
+    q, k = qbuf[:, :, :heads], kbuf[:, :, :heads]
+    untouched = kbuf[:, :, heads:].clone()
+    qo, ko = h3a.qk_norm_rope(q, k, _dev(d["gamma_q"]), _dev(d["gamma_k"]), grid, THETA, EPS, inplace=True)
+    torch.cuda.synchronize()
+    assert qo.data_ptr() == q.data_ptr()
+    for x, g, out in ((d["q"], d["gamma_q"], qo), (d["k"], d["gamma_k"], ko)):
+        want = orc.qk_norm_rope_bf16(x[:, :, :heads].contiguous(), g.numpy(), grid, THETA, EPS)
+        check_prologue(bits(out), want, "strided")
+    assert torch.equal(kbuf[:, :, heads:], untouched)
+
+
+# ---------------------------------------------------------------- router
+
+ROUTER_CASES = [
+    ("tiny", 1, 2, (2, 4, 8), 0.75),             # one block: k = 1
+    ("layer8k", 1, 56, (8, 24, 42), 0.75),       # 63 blocks, k = 16
+    ("ragged", 2, 3, (3, 7, 55), 0.6),           # 1155 tokens: 10 blocks, tail of 3
+    ("k_all", 1, 4, (4, 16, 40), 0.0),           # k = nblk
+]
+
+
+@pytest.mark.parametrize("name,B,heads,grid,s", ROUTER_CASES, ids=[c[0] for c in ROUTER_CASES])
+def test_router_parity(orc, name, B, heads, grid, s):
+    d = _inputs(B, heads, grid, "structured" if name != "tiny" else "normal")
+    qb = orc.qk_norm_rope_bf16(d["q"], d["gamma_q"].numpy(), grid)
+    kb = orc.qk_norm_rope_bf16(d["k"], d["gamma_k"].numpy(), grid)
+    idx = h3a.route(_dev(from_bits(qb)), _dev(from_bits(kb)), s)
+    torch.cuda.synchronize()
+    ora_idx, ora_sc = orc.route(qb, kb, s)
+    check_router(idx.cpu().numpy(), ora_idx, ora_sc, name)
+
+
+def test_router_exact_ties_pick_lower_index(orc):
+    """Key blocks that are exact copies score identically; the lower index wins."""
+    grid = (4, 8, 16)                      # 512 tokens, 4 blocks
+    d = _inputs(1, 2, grid)
+    k = d["k"].clone()
+    k[:, 256:384] = k[:, 0:128]            # block 2 == block 0
+    k[:, 384:512] = k[:, 128:256]          # block 3 == block 1
+    q = d["q"]
+    for s in (0.75, 0.5):
+        idx = h3a.route(_dev(q), _dev(k), s).cpu().numpy()
+        ora_idx, ora_sc = orc.route(q, k, s)
+        np.testing.assert_array_equal(idx, ora_idx)
+        assert (idx < 2).all()             # never the later copies
+
+
+# ---------------------------------------------------------------- attention
+
+ATTN_CASES = [
+    ("tiny", 1, 2, (2, 4, 8)),               # N = 64 < one tile
+    ("one_block", 1, 3, (2, 8, 8)),          # N = 128
+    ("tail1", 1, 2, (1, 1, 257)),            # N = 257: a tail of one token
+    ("ragged", 2, 3, (3, 11, 13)),           # N = 429, B = 2
+    ("odd_tiles", 1, 2, (5, 8, 16)),         # N = 640: 5 tiles, the last pair has one tile
+]
+
+
+@pytest.mark.parametrize("name,B,heads,grid", ATTN_CASES, ids=[c[0] for c in ATTN_CASES])
+def test_dense_attention_parity(orc, name, B, heads, grid):
+    d = _inputs(B, heads, grid, "normal")
+    o = h3a.attention(_dev(d["q"]), _dev(d["k"]), _dev(d["v"]))
+    torch.cuda.synchronize()
+    assert h3a.last_device_error() == 0
+    N = grid[0] * grid[1] * grid[2]
+    rows = np.arange(B * heads * N)
+    want = orc.attention_rows(d["q"], d["k"], d["v"], rows)
+    check_attention(gather_rows(o, rows), want, name)
+
+
+@pytest.mark.parametrize("name,B,heads,grid", ATTN_CASES[2:], ids=[c[0] for c in ATTN_CASES[2:]])
+@pytest.mark.parametrize("s", [0.5, 0.8])
+def test_sparse_attention_parity(orc, name, B, heads, grid, s):
+    d = _inputs(B, heads, grid, "structured")
+    ora_idx, _ = orc.route(d["q"], d["k"], s)
+    o = h3a.attention(_dev(d["q"]), _dev(d["k"]), _dev(d["v"]), _dev(torch.from_numpy(ora_idx)))
+    torch.cuda.synchronize()
+    assert h3a.last_device_error() == 0
+    N = grid[0] * grid[1] * grid[2]
+    rows = np.arange(B * heads * N)
+    want = orc.attention_rows(d["q"], d["k"], d["v"], rows, ora_idx)
+    check_attention(gather_rows(o, rows), want, f"{name}-s{s}")
+
+
+def test_sparse_with_every_block_equals_dense_bitwise():
+    grid, heads = (4, 16, 40), 3                 # 2560 tokens, 20 blocks
+    d = _inputs(1, heads, grid, "structured")
+    q, k, v = (_dev(d[n]) for n in "qkv")
+    nblk = 20
+    all_blocks = torch.arange(nblk, dtype=torch.int32).expand(1, heads, nblk, nblk).contiguous()
+    dense = h3a.attention(q, k, v)
+    sparse = h3a.attention(q, k, v, all_blocks.cuda())
+    torch.cuda.synchronize()
+    assert torch.equal(dense, sparse)
+
+
+def test_identical_keys_give_mean_value():
+    """All keys equal: every query sees uniform weights, so O = mean(V) per head."""
+    grid, heads = (4, 32, 32), 4                 # 4096 tokens
+    d = _inputs(1, heads, grid)
+    k = d["k"][:, :1].expand(-1, 4096, -1, -1).contiguous()
+    o = h3a.attention(_dev(d["q"]), _dev(k), _dev(d["v"]))
+    torch.cuda.synchronize()
+    mean_v = d["v"].double().mean(dim=1)         # [1, heads, 96]
+    err = (o.cpu().double() - mean_v[:, None]).abs().max().item()
+    assert err <= 2e-3, err
+
+
+def test_dense_attention_layer8k_sampled(orc):
+    d = synth.draw_workload("layer8k")
+    o = h3a.attention(_dev(d["q"]), _dev(d["k"]), _dev(d["v"]))
+    torch.cuda.synchronize()
+    rows = synth.sample_rows(1, 56, 8064, 4096).numpy()
+    want = orc.attention_rows(d["q"], d["k"], d["v"], rows)
+    check_attention(gather_rows(o, rows), want, "layer8k")

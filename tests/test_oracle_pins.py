@@ -432,3 +432,26 @@ def test_sparse_single_block_is_dense_on_that_block(orc):
         L = qf[n] @ kf[keys].T / math.sqrt(D)
         w = np.exp(L - L.max())
         np.testing.assert_allclose(out[n], (w / w.sum()) @ vf[keys], rtol=0, atol=1e-12)
+
+
+def test_round_bf16_nearest_even_from_fp64(orc):
+    """Rounding is taken once, straight from fp64: halfway cases go to even, and
+    1 + 2^-8 + 2^-30 (just above halfway) rounds up -- a detour through fp32
+    would round it to the halfway point first and then down to even."""
+    x = np.array([1.0, 1 + 2 ** -8, 1 + 1.5 * 2 ** -8, 1 + 2 ** -9, 1 + 2 ** -8 + 2 ** -30, -3.14159,
+                  1e-40, 3.4e38, 3.39e38, 0.0, 1.5 * 2 ** -133])
+    got = orc.round_bf16(x).tolist()
+    assert got == [0x3F80, 0x3F80, 0x3F81, 0x3F80, 0x3F81, 0xC049, 0x0001, 0x7F80, 0x7F7F, 0x0000, 0x0002]
+
+
+def test_prologue_variants_agree(orc):
+    """The token-subset and bf16-output forms restate the same per-token steps."""
+    rng = np.random.default_rng(15)
+    grid = (2, 3, 5)
+    x = _bf16(rng.normal(size=(2, 30, 3, D)))
+    g = (1 + 0.1 * rng.normal(size=D)).astype(np.float32)
+    full = orc.qk_norm_rope(x, g, grid)
+    toks = np.array([0, 7, 29, 30, 59])
+    sub = orc.qk_norm_rope_tokens(x, g, grid, toks)
+    np.testing.assert_array_equal(sub, full.reshape(60, 3, D)[toks])
+    np.testing.assert_array_equal(orc.qk_norm_rope_bf16(x, g, grid), orc.round_bf16(full))
