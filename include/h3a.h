@@ -156,6 +156,15 @@ h3a_status h3a_selftest_wait_timeout(uint32_t limit_us, h3a_stream_t stream);
 h3a_status h3a_selftest_mma(const void* a, const void* b, float* s_out, float* r_out,
                             h3a_stream_t stream);
 
+/* Self-check of the exponentials of the attention softmax (no counterpart on
+ * the pages): y[i] = 2^x[i] for n device floats, computed by the same device
+ * code the softmax uses -- the FMA-pipe polynomial (use_poly != 0: Cody-Waite
+ * split x = n + f with f in [-1/2, 1/2], degree-3 minimax polynomial for 2^f,
+ * max relative error 7.5e-5 for x >= -125; x below -126 is clamped there and
+ * yields at most 2^-125) or ex2.approx (use_poly == 0).  Asynchronous on
+ * `stream`.  INVALID_ARG for n < 0 or null / misaligned pointers. */
+h3a_status h3a_selftest_exp2(const float* x, float* y, int32_t n, int32_t use_poly, h3a_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

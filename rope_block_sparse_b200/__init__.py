@@ -10,7 +10,7 @@ All compute runs in libh3a.so (include/h3a.h); the Python layer only marshals
 arguments.  ``synth`` holds the seeded synthetic input generators.
 """
 from .h3a import (H3AError, attention, attention_core, last_device_error, load, qk_norm_rope, route,
-                  route_k, route_workspace_size, selftest_mma, selftest_wait_timeout)
+                  route_k, route_workspace_size, selftest_exp2, selftest_mma, selftest_wait_timeout)
 
 __all__ = ["H3AError", "attention", "attention_core", "last_device_error", "load", "qk_norm_rope", "route",
-           "route_k", "route_workspace_size", "selftest_mma", "selftest_wait_timeout"]
+           "route_k", "route_workspace_size", "selftest_exp2", "selftest_mma", "selftest_wait_timeout"]

@@ -261,4 +261,11 @@ h3a_status h3a_selftest_mma(const void* a, const void* b, float* s_out, float* r
     return e == cudaSuccess ? H3A_OK : cuda_fail(e);
 }
 
+h3a_status h3a_selftest_exp2(const float* x, float* y, int32_t n, int32_t use_poly, h3a_stream_t stream) {
+    if (n < 0 || (n > 0 && (!x || !y))) return H3A_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(x) & 3u) || (reinterpret_cast<uintptr_t>(y) & 3u)) return H3A_ERR_INVALID_ARG;
+    cudaError_t e = launch_selftest_exp2(x, y, n, use_poly ? 1 : 0, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? H3A_OK : cuda_fail(e);
+}
+
 }  // extern "C"

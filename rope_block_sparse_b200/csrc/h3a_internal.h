@@ -38,6 +38,7 @@ cudaError_t launch_attention(const CUtensorMap& tq, const CUtensorMap& tk, const
 
 // Self-checks (selftest.cu).
 cudaError_t launch_selftest_wait(uint64_t limit_ns, int* status, cudaStream_t st);
+cudaError_t launch_selftest_exp2(const float* x, float* y, int n, int poly, cudaStream_t st);
 cudaError_t launch_selftest_mma(const CUtensorMap& ta, const CUtensorMap& tb, float* s_out, float* r_out,
                                 int* status, uint64_t timeout_ns, cudaStream_t st);
 

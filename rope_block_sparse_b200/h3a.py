@@ -25,7 +25,7 @@ STATUS_NAMES = {0: "H3A_OK", 1: "H3A_ERR_INVALID_ARG", 2: "H3A_ERR_UNSUPPORTED",
 # Every function the header declares; checked by the ABI test.
 EXPORTS = ("h3a_qk_norm_rope", "h3a_route_k", "h3a_route_workspace_size", "h3a_route", "h3a_attention",
            "h3a_status_string", "h3a_last_cuda_error_string", "h3a_last_device_error",
-           "h3a_selftest_wait_timeout", "h3a_selftest_mma")
+           "h3a_selftest_wait_timeout", "h3a_selftest_mma", "h3a_selftest_exp2")
 
 
 class H3AError(RuntimeError):
@@ -82,6 +82,8 @@ def load() -> ctypes.CDLL:
     lib.h3a_selftest_wait_timeout.restype = st
     lib.h3a_selftest_mma.argtypes = [P, P, P, P, P]
     lib.h3a_selftest_mma.restype = st
+    lib.h3a_selftest_exp2.argtypes = [P, P, i32, i32, P]
+    lib.h3a_selftest_exp2.restype = st
     _lib = lib
     return lib
 
@@ -222,6 +224,16 @@ def selftest_mma(a: torch.Tensor, b: torch.Tensor):
     r = torch.empty((128, HEAD_DIM), dtype=torch.float32, device=a.device)
     _check("h3a_selftest_mma", lib.h3a_selftest_mma(_ptr(a), _ptr(b), _ptr(s), _ptr(r), _stream_handle()))
     return s, r
+
+
+def selftest_exp2(x: torch.Tensor, use_poly: bool = True) -> torch.Tensor:
+    """2^x by the softmax's exponential (FMA-pipe polynomial, or ex2.approx): fp32 CUDA tensor in and out."""
+    lib = load()
+    if not x.is_cuda or x.dtype != torch.float32 or not x.is_contiguous():
+        raise ValueError("x must be a contiguous fp32 CUDA tensor")
+    y = torch.empty_like(x)
+    _check("h3a_selftest_exp2", lib.h3a_selftest_exp2(_ptr(x), _ptr(y), x.numel(), int(use_poly), _stream_handle()))
+    return y
 
 
 def attention_core(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, gamma_q: torch.Tensor,

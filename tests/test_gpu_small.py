@@ -196,3 +196,21 @@ def test_dense_attention_layer8k_sampled(orc):
     rows = synth.sample_rows(1, 56, 8064, 4096).numpy()
     want = orc.attention_rows(d["q"], d["k"], d["v"], rows)
     check_attention(gather_rows(o, rows), want, "layer8k")
+
+
+def test_polynomial_exp2_within_its_bound():
+    """The FMA-pipe exp2 of the softmax against 2^x (fp64): relative error at most
+    8e-5 wherever the result is a normal float (x >= -125); below that it yields
+    at most 2^-125 (P is zero there for bf16 purposes).  ex2.approx is checked
+    alongside at the bound CUDA documents for it (2 ulp, here 2^-22 relative)."""
+    g = torch.Generator().manual_seed(5)
+    x = torch.cat([torch.rand(1 << 20, generator=g) * 140.0 - 130.0,
+                   torch.tensor([0.0, 0.5, -0.5, 1.0, -1.0, 8.0, -125.0, -126.0, -127.5, -1e4, float("-inf")])])
+    want = torch.exp2(x.double())
+    for poly, bound in ((True, 8e-5), (False, 2.0 ** -22)):
+        y = h3a.selftest_exp2(x.cuda(), use_poly=poly).cpu().double()
+        normal = x >= -125.0
+        rel = ((y[normal] - want[normal]).abs() / want[normal]).max().item()
+        assert rel <= bound, (poly, rel)
+        assert (y[~normal].abs() <= 2.0 ** -125).all()
+        assert (y >= 0).all()
