@@ -106,6 +106,30 @@ h3a_status h3a_route(const void* q, const void* k, const h3a_qkv_desc* d, double
                      int32_t block, int32_t* block_idx, int64_t* k_out, void* workspace,
                      size_t ws_bytes, h3a_stream_t stream);
 
+/* Capacity of the scratch built into h3a_route_noalloc: 64 MiB, enough for
+ * B * heads * ceil(N / 128) <= 87,381 (e.g. 56 heads of a 124,992-token clip). */
+#define H3A_ROUTE_NOALLOC_MAX_BYTES ((size_t)64 << 20)
+
+/* h3a_route for callers that cannot allocate device memory (no counterpart on
+ * the pages).  Some callers have no allocator at hand where they route -- an
+ * embedding runtime that hands out none after start-up, code inside a host
+ * callback or another allocator's critical section, a serving loop with a
+ * fixed memory budget -- so this variant takes no workspace: its scratch is a
+ * file-scope device array of H3A_ROUTE_NOALLOC_MAX_BYTES that every GPU
+ * loading the library holds until process exit.  It calls no cudaMalloc,
+ * cudaFree or other allocating routine.  Arguments and results are those of
+ * h3a_route.
+ * The first call on a device resolves the array's device address for that
+ * device (cudaGetSymbolAddress with the device current): make that first call
+ * before any stream capture.  Every call shares the one array and overwrites
+ * what it reads, so nothing needs clearing, but calls whose executions overlap
+ * on the GPU (other streams, other host threads) race on it.
+ * Errors: those of h3a_route; H3A_ERR_WORKSPACE when the shape needs more than
+ * H3A_ROUTE_NOALLOC_MAX_BYTES of scratch (h3a_route_workspace_size bytes);
+ * H3A_ERR_CUDA if the set-up fails. */
+h3a_status h3a_route_noalloc(const void* q, const void* k, const h3a_qkv_desc* d, double sparsity,
+                             int32_t block, int32_t* block_idx, int64_t* k_out, h3a_stream_t stream);
+
 /* Bidirectional attention O = softmax(scale * Q K^T) V per (b, head).
  * Source: dense lossless path of the news.cocoloop.cn MiniMax-H3 SGLang
  * report (opening quote: no approximation; SSIM 1.0000) and its SubBlock

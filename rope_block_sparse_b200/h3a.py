@@ -25,7 +25,8 @@ STATUS_NAMES = {0: "H3A_OK", 1: "H3A_ERR_INVALID_ARG", 2: "H3A_ERR_UNSUPPORTED",
 # Every function the header declares; checked by the ABI test.
 EXPORTS = ("h3a_qk_norm_rope", "h3a_route_k", "h3a_route_workspace_size", "h3a_route", "h3a_attention",
            "h3a_status_string", "h3a_last_cuda_error_string", "h3a_last_device_error",
-           "h3a_selftest_wait_timeout", "h3a_selftest_mma", "h3a_selftest_exp2")
+           "h3a_selftest_wait_timeout", "h3a_selftest_mma", "h3a_selftest_exp2", "h3a_route_noalloc")
+ROUTE_NOALLOC_MAX_BYTES = 64 << 20  # H3A_ROUTE_NOALLOC_MAX_BYTES
 
 
 class H3AError(RuntimeError):
@@ -84,6 +85,8 @@ def load() -> ctypes.CDLL:
     lib.h3a_selftest_mma.restype = st
     lib.h3a_selftest_exp2.argtypes = [P, P, i32, i32, P]
     lib.h3a_selftest_exp2.restype = st
+    lib.h3a_route_noalloc.argtypes = [P, P, ctypes.POINTER(QkvDesc), f64, i32, P, ctypes.POINTER(ctypes.c_int64), P]
+    lib.h3a_route_noalloc.restype = st
     _lib = lib
     return lib
 
