@@ -9,48 +9,43 @@
 // 2p and 2p+1, i.e. the router's query blocks -- and streams 128-row K/V tiles
 // through shared memory: every KV block for dense attention, or each tile's
 // own routed list in sparse mode (a KV tile both lists name at the same step is
-// loaded once and shared).  Each 128-key block is processed as two 64-key
-// half-steps u = 2j + h.  Warp roles (384 threads):
+// loaded once and shared).  Warp roles (384 threads):
 //   warp 0      TMA producer: Q tiles once, then a 3-stage K ring and a 3-stage
 //               V ring (64-byte swizzled 128 x 32 chunks, 3 per 128 x 96 tile).
 //   warp 1      owns tensor memory (512 columns) and issues tcgen05.mma from one
-//               thread: S_t[h] = Q_t K_h^T (M=128, N=64, K=96 as 6 steps of 16)
-//               into one of two S buffers per tile, O_t += P_t[h] V_h (M=128,
-//               N=96, K=64 as 4 steps; P read from TMEM, V as an MN-major
-//               operand).  Order per half-step u and tile t: wait P_t(u),
-//               PV_t(u), then QK_t(u+2) into the buffer PV_t(u) just read, so
-//               the next S of every tile is computed while its softmax runs.
+//               thread: S_t = Q_t K^T (M=128, N=128, K=96 as 6 steps of 16) into
+//               TMEM, O_t += P_t V (M=128, N=96, K=128 as 8 steps, P read from
+//               TMEM, V as an MN-major operand).  Order per step j:
+//               PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1), so each softmax group
+//               waits only on its own tile's chain.
 //   warps 4-7   softmax of tile 0, warps 8-11 softmax of tile 1: thread r owns
-//               query row r (TMEM lane r); it reads its 64 S values from TMEM,
-//               keeps the running max / sum in fp32 (log2 domain), computes
-//               exponentials on the MUFU unit and, for three pairs in eight, as
-//               a polynomial on the FMA pipe, writes P as packed bf16 over the
-//               first 32 columns of the S buffer, and rescales its O row in TMEM
-//               only when the max grew by more than 2^8 (the final division by
-//               the row sum keeps this exact).  At the end it divides O by the
-//               row sum, rounds once to bf16 and stores the row.
-// TMEM columns: S_0[0..1] [0,128), S_1[0..1] [128,256), O_0 [256,352),
-// O_1 [352,448).  Every mbarrier wait is bounded (timeout + CTA abort flag); a
-// timeout sets the device status word instead of hanging or trapping.
+//               query row r (TMEM lane r); it reads its S row from TMEM, keeps
+//               the running max / sum in fp32 (log2 domain, exp2), writes P as
+//               packed bf16 over the first 64 columns of S, and rescales its O
+//               row in TMEM only when the max grew by more than 2^8 (the final
+//               division by the row sum keeps this exact).  At the end it divides
+//               O by the row sum, rounds once to bf16 and stores the row.
+// TMEM columns: S_0 [0,128), S_1 [128,256), O_0 [256,352), O_1 [352,448).
+// Every mbarrier wait is bounded (timeout + CTA abort flag); a timeout sets the
+// device status word instead of hanging or trapping.
 #include <cuda_bf16.h>
 
 #include "h3a_internal.h"
-#include "fastmath.cuh"
 #include "sm100.cuh"
 
 namespace h3a {
 namespace {
 
-constexpr int kThreads = 384;
+constexpr int kSoftmaxWarps = 16;                  // 4 warpgroups: (tile, column half)
+constexpr int kProducerWarp = 16, kMmaWarp = 17;
+constexpr int kThreads = 32 * (kSoftmaxWarps + 2);  // 576
 constexpr int kStages = 3;
 constexpr int kChunkBytes = 128 * 64;        // 128 rows x 32 bf16, 64-byte swizzle
 constexpr int kTileBytes = 3 * kChunkBytes;  // 128 x 96 bf16
-constexpr int kHalf = 64;                     // keys per half-step (half a 128-token KV block)
 constexpr uint32_t kTmemCols = 512;
-// TMEM columns: S_t[h] (64 fp32 columns; P_t[h] as packed bf16 over its first
-// 32) at 128t + 64h, O_t (96 fp32 columns) at 256 + 96t.
-__host__ __device__ constexpr uint32_t col_s(int t, int h) { return 128u * t + 64u * h; }
-__host__ __device__ constexpr uint32_t col_o(int t) { return 256u + 96u * t; }
+// TMEM column of S_t / O_t
+__host__ __device__ constexpr uint32_t col_s(int t) { return t ? 128u : 0u; }
+__host__ __device__ constexpr uint32_t col_o(int t) { return t ? 352u : 256u; }
 constexpr uint32_t kSwizzle64 = 4;
 
 struct AttnSmem {
@@ -60,9 +55,12 @@ struct AttnSmem {
     uint64_t q_full[2];
     uint64_t k_full[kStages], k_empty[kStages];
     uint64_t v_full[kStages], v_empty[kStages];
-    uint64_t s_full[2][2], p_full[2][2];  // [tile][S buffer]
-    uint64_t pv_done[2], o_done[2];
+    uint64_t s_full[2], p_full[2], o_done[2];
+    uint64_t xbar[2][2];         // [buffer][tile]: half-row maxima exchanged
+    uint64_t lbar[2];            // [tile]: half-row sums exchanged at the end
     uint64_t mma_drain;
+    float xmax[2][2][2][128];    // [buffer][tile][half][row]
+    float lsum[2][2][128];       // [tile][half][row]
     uint32_t tmem_base;
     int abort_flag;
     int never;  // stays 0: abort flag for waits that must ignore an abort
@@ -85,17 +83,30 @@ __device__ __forceinline__ void raise_timeout(const AttnArgs& a, volatile int* a
     atomicOr(a.status, kDevTimeout);
 }
 
-// K-major operand from a 128 x 96 tile (three swizzled 32-column chunks of
-// 64-byte rows): k-step s covers columns [16s, 16s + 16), starting at row0.
-__device__ __forceinline__ uint64_t kmajor_desc(const uint8_t* tile, int s, int row0) {
-    return smem_desc(smem_u32(tile) + (s >> 1) * kChunkBytes + (s & 1) * 32 + row0 * 64, 16, 512, kSwizzle64);
+// Shared-memory descriptors are built once per buffer; a k-step or a ring
+// stage only moves the start address, i.e. adds a constant (in 16-byte units)
+// to the low field (addresses stay below 2^18, so the 14-bit field never
+// carries).  This keeps the single MMA-issuing thread at a few instructions
+// per tcgen05.mma -- computing descriptors per MMA made the issue thread,
+// not the tensor core, the bottleneck.
+//
+// K-major 128 x 96 tile (three swizzled 32-column chunks of 64-byte rows):
+// k-step s covers columns [16s, 16s + 16).
+__device__ __forceinline__ uint64_t kmajor_base(const uint8_t* tile) {
+    return smem_desc(smem_u32(tile), 16, 512, kSwizzle64);
+}
+__host__ __device__ constexpr uint32_t kmajor_step(int s) {
+    return static_cast<uint32_t>(((s >> 1) * kChunkBytes + (s & 1) * 32) >> 4);
 }
 
 // The same [128 kv rows x 96] tile read as an MN-major operand (N = 96 along
-// the contiguous dimension, K = kv rows): 16 rows from row0.
-__device__ __forceinline__ uint64_t mnmajor_desc(const uint8_t* tile, int row0) {
-    return smem_desc(smem_u32(tile) + row0 * 64, kChunkBytes, 512, kSwizzle64);
+// the contiguous dimension, K = kv rows): k-step s covers rows [16s, 16s + 16).
+__device__ __forceinline__ uint64_t mnmajor_base(const uint8_t* tile) {
+    return smem_desc(smem_u32(tile), kChunkBytes, 512, kSwizzle64);
 }
+__host__ __device__ constexpr uint32_t mnmajor_step(int s) { return static_cast<uint32_t>((s * 16 * 64) >> 4); }
+
+constexpr uint32_t kStageStep = kTileBytes >> 4;  // descriptor distance between ring stages
 
 struct KvPlan {
     int kv0, kv1;
@@ -172,106 +183,100 @@ __device__ void producer(AttnSmem& sm, const AttnArgs& a, const CUtensorMap* tq,
     }
 }
 
-// ---------------------------------------------------------------- MMA issue
-
 struct MmaState {
-    uint32_t ks = 0, kph = 0, vs = 0, vph = 0;  // ring positions
-    uint32_t kst[2] = {0, 0}, vst[2] = {0, 0};  // stage each tile reads for the current block
+    uint32_t ks = 0, kph = 0, vs = 0, vph = 0;
+    uint32_t k_stage_t0 = 0, v_stage_t0 = 0;
+    uint64_t dq[2], dk, dv;  // base descriptors: Q tiles, K stage 0, V stage 0
 };
 
-// S_t[h] = Q_t K_half^T for half h of the step's KV block (M=128, N=64, K=96).
 __device__ __forceinline__ bool issue_qk(AttnSmem& sm, const AttnArgs& a, MmaState& st, uint32_t tmem, int t,
-                                         int u, const KvPlan& p, volatile int* abort_flag) {
-    const int h = u & 1;
-    if (h == 0) {
-        if (t == 0 || !p.shared) {
-            if (!mbar_wait(&sm.k_full[st.ks], st.kph, abort_flag, a.timeout_ns)) return false;
-            st.kst[t] = st.ks;
-            if (++st.ks == kStages) {
-                st.ks = 0;
-                st.kph ^= 1u;
-            }
-        } else {
-            st.kst[1] = st.kst[0];
+                                         const KvPlan& p, volatile int* abort_flag) {
+    uint32_t stage;
+    if (t == 0 || !p.shared) {
+        if (!mbar_wait(&sm.k_full[st.ks], st.kph, abort_flag, a.timeout_ns)) return false;
+        stage = st.ks;
+        if (++st.ks == kStages) {
+            st.ks = 0;
+            st.kph ^= 1u;
         }
+    } else {
+        stage = st.k_stage_t0;
     }
-    const uint32_t stage = st.kst[t];
+    if (t == 0) st.k_stage_t0 = stage;
     tc_fence_after_sync();
-    constexpr uint32_t idesc = idesc_bf16_f32(128, kHalf, 0, 0);
+    constexpr uint32_t idesc = idesc_bf16_f32(128, 128, 0, 0);
+    const uint64_t dq = st.dq[t];
+    const uint64_t dk = st.dk + stage * kStageStep;
+    const uint32_t d = tmem + col_s(t);
 #pragma unroll
-    for (int s = 0; s < 6; ++s)
-        mma_ss(tmem + col_s(t, h), kmajor_desc(sm.q[t], s, 0), kmajor_desc(sm.k[stage], s, kHalf * h), idesc,
-               s > 0 ? 1u : 0u);
-    tc_commit(&sm.s_full[t][h]);
-    if (h == 1 && (t == 1 || !p.shared)) tc_commit(&sm.k_empty[stage]);
+    for (int s = 0; s < 6; ++s) mma_ss(d, dq + kmajor_step(s), dk + kmajor_step(s), idesc, s > 0 ? 1u : 0u);
+    tc_commit(&sm.s_full[t]);
+    if (t == 1 || !p.shared) tc_commit(&sm.k_empty[stage]);
     return true;
 }
 
-// O_t += P_t[h] V_half (M=128, N=96, K=64), P read from TMEM.
 __device__ __forceinline__ bool issue_pv(AttnSmem& sm, const AttnArgs& a, MmaState& st, uint32_t tmem, int t,
-                                         int u, const KvPlan& p, volatile int* abort_flag) {
-    const int h = u & 1;
-    if (h == 0) {
-        if (t == 0 || !p.shared) {
-            if (!mbar_wait(&sm.v_full[st.vs], st.vph, abort_flag, a.timeout_ns)) return false;
-            st.vst[t] = st.vs;
-            if (++st.vs == kStages) {
-                st.vs = 0;
-                st.vph ^= 1u;
-            }
-        } else {
-            st.vst[1] = st.vst[0];
+                                         const KvPlan& p, bool first, volatile int* abort_flag) {
+    uint32_t stage;
+    if (t == 0 || !p.shared) {
+        if (!mbar_wait(&sm.v_full[st.vs], st.vph, abort_flag, a.timeout_ns)) return false;
+        stage = st.vs;
+        if (++st.vs == kStages) {
+            st.vs = 0;
+            st.vph ^= 1u;
         }
+    } else {
+        stage = st.v_stage_t0;
     }
-    const uint32_t stage = st.vst[t];
+    if (t == 0) st.v_stage_t0 = stage;
     tc_fence_after_sync();
     constexpr uint32_t idesc = idesc_bf16_f32(128, 96, 0, 1);
+    const uint64_t dv = st.dv + stage * kStageStep;
+    const uint32_t d = tmem + col_o(t), pa = tmem + col_s(t);
+    // keys 0..63: P at S columns [0, 32); keys 64..127: P at S columns [64, 96)
+    mma_ts(d, pa, dv, idesc, first ? 0u : 1u);
 #pragma unroll
-    for (int s = 0; s < kHalf / 16; ++s)
-        mma_ts(tmem + col_o(t), tmem + col_s(t, h) + 8 * s, mnmajor_desc(sm.v[stage], kHalf * h + 16 * s), idesc,
-               (u == 0 && s == 0) ? 0u : 1u);
-    tc_commit(&sm.pv_done[t]);
-    if (h == 1 && (t == 1 || !p.shared)) tc_commit(&sm.v_empty[stage]);
+    for (int s = 1; s < 8; ++s) mma_ts(d, pa + 64 * (s >> 2) + 8 * (s & 3), dv + mnmajor_step(s), idesc, 1u);
+    if (t == 1 || !p.shared) tc_commit(&sm.v_empty[stage]);
     return true;
 }
 
-// Issue order over half-steps u = 2j + h: QK for u = 0, 1 of both tiles, then
-// per u and tile: wait P_t(u), PV_t(u), QK_t(u + 2) into the S buffer PV_t(u)
-// has just consumed (tcgen05.mma from one thread executes in issue order).
-// Each tile therefore always has the next S ready while its softmax runs.
 __device__ void mma_issuer(AttnSmem& sm, const AttnArgs& a, uint32_t tmem, bool has1, const int32_t* l0,
                            const int32_t* l1, volatile int* abort_flag) {
     const int ntiles = has1 ? 2 : 1;
-    const int nsub = 2 * a.n_iter;
+    MmaState st;
+    st.dq[0] = kmajor_base(sm.q[0]);
+    st.dq[1] = kmajor_base(sm.q[1]);
+    st.dk = kmajor_base(sm.k[0]);
+    st.dv = mnmajor_base(sm.v[0]);
     bool ok = true;
     for (int t = 0; t < ntiles && ok; ++t) ok = mbar_wait(&sm.q_full[t], 0u, abort_flag, a.timeout_ns);
-    MmaState st;
-    KvPlan cur = kv_plan(l0, l1, has1, 0);
-    for (int u = 0; u < 2 && ok; ++u)
-        for (int t = 0; t < ntiles && ok; ++t) ok = issue_qk(sm, a, st, tmem, t, u, cur, abort_flag);
-    KvPlan next = cur;
-    for (int u = 0; u < nsub && ok; ++u) {
-        const int h = u & 1;
-        if (h == 0) {
-            cur = (u == 0) ? cur : next;
-            if (u + 2 < nsub) next = kv_plan(l0, l1, has1, (u >> 1) + 1);
-        }
+    // block lists are read one step ahead so their load latency stays off the issue path
+    KvPlan p = kv_plan(l0, l1, has1, 0);
+    KvPlan pn = a.n_iter > 1 ? kv_plan(l0, l1, has1, 1) : p;
+    if (ok)
+        for (int t = 0; t < ntiles && ok; ++t) ok = issue_qk(sm, a, st, tmem, t, p, abort_flag);
+    for (int j = 0; j < a.n_iter && ok; ++j) {
+        const bool more = j + 1 < a.n_iter;
+        const KvPlan pnn = (j + 2 < a.n_iter) ? kv_plan(l0, l1, has1, j + 2) : pn;
         for (int t = 0; t < ntiles && ok; ++t) {
-            if (!mbar_wait(&sm.p_full[t][h], static_cast<uint32_t>((u >> 1) & 1), abort_flag, a.timeout_ns)) {
+            if (!mbar_wait(&sm.p_full[t], static_cast<uint32_t>(j & 1), abort_flag, a.timeout_ns)) {
                 ok = false;
                 break;
             }
             tc_fence_after_sync();
-            if (!issue_pv(sm, a, st, tmem, t, u, cur, abort_flag)) {
+            if (!issue_pv(sm, a, st, tmem, t, p, j == 0, abort_flag)) {
                 ok = false;
                 break;
             }
-            if (u + 2 < nsub) {
-                if (!issue_qk(sm, a, st, tmem, t, u + 2, next, abort_flag)) ok = false;
-            } else if (u == nsub - 1) {
+            if (more) {
+                if (!issue_qk(sm, a, st, tmem, t, pn, abort_flag)) ok = false;
+            } else {
                 tc_commit(&sm.o_done[t]);
             }
         }
+        p = pn;
+        pn = pnn;
     }
     if (!ok) raise_timeout(a, abort_flag);
     // Drain: every MMA issued must have completed before TMEM is released.
@@ -280,36 +285,50 @@ __device__ void mma_issuer(AttnSmem& sm, const AttnArgs& a, uint32_t tmem, bool 
     mbar_wait(&sm.mma_drain, 0u, never, a.timeout_ns);
 }
 
-// ---------------------------------------------------------------- softmax
+// Exponentials of one 64-key half row with reference m: P packed to bf16 into
+// the first 32 columns of this half's S region; returns the partial sums.
+__device__ __forceinline__ float exp_store_half(const uint32_t (&s)[2][32], float c, float m, uint32_t tS,
+                                                float* hmax) {
+    const float neg_m = -m;
+    float pm[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+    float ps[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int q2 = 0; q2 < 2; ++q2) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const float x0 = __uint_as_float(s[q2][2 * i]), x1 = __uint_as_float(s[q2][2 * i + 1]);
+            if (hmax) pm[i & 3] = fmaxf(pm[i & 3], fmaxf(x0, x1));
+            const float p0 = ex2_approx(fmaf(x0, c, neg_m));
+            const float p1 = ex2_approx(fmaf(x1, c, neg_m));
+            ps[i & 3] += p0 + p1;
+            pk[i] = pack_bf16x2(p0, p1);
+        }
+        tmem_st_x16(tS + 16 * q2, pk);
+    }
+    if (hmax) *hmax = fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3]));
+    return (ps[0] + ps[1]) + (ps[2] + ps[3]);
+}
 
-// Pairs i (mod 8) whose exponentials take the polynomial path; the rest use
-// ex2.approx on the MUFU unit.  Three of eight pairs splits the exponentials
-// between the two pipes so that neither bounds the step before the tensor core.
-#ifndef H3A_POLY_PAIRS
-#define H3A_POLY_PAIRS 0x94u
-#endif
-constexpr uint32_t kPolyPairs = H3A_POLY_PAIRS;
-
-__device__ void softmax_group(AttnSmem& sm, const AttnArgs& a, uint32_t tmem, int t, int b, int h, int qb,
+// Softmax of query tile t, key columns [64*hf, 64*hf + 64) of every 128-key
+// block: thread r owns row r (TMEM lane r) of that half.  The two halves of a
+// row run in two warpgroups and agree on the row's reference max through
+// shared memory and a bounded mbarrier wait per block.
+__device__ void softmax_group(AttnSmem& sm, const AttnArgs& a, uint32_t tmem, int t, int hf, int b, int h, int qb,
                               const int32_t* list, volatile int* abort_flag) {
     const int lane = threadIdx.x & 31;
     const int quarter = (threadIdx.x >> 5) & 3;  // TMEM lanes [32*quarter, 32*quarter + 32)
     const int row = quarter * 32 + lane;
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
-    const uint32_t tO = tmem + lane_addr + col_o(t);
+    const uint32_t tS = tmem + lane_addr + col_s(t) + 64u * hf;
+    const uint32_t tO = tmem + lane_addr + col_o(t) + 48u * hf;
     const float c = a.scale_log2;
-    const uint64_t c2 = f2(c, c);
-    const int nsub = 2 * a.n_iter;
-    float m_used = -INFINITY;  // running max of scaled logits (log2 units) used for P
-    uint64_t l2 = f2(0.f, 0.f);  // running sum of P, two partial lanes
-    int kv = 0;
+    float m_used = -INFINITY;  // row reference max of scaled logits (log2 units)
+    float l = 0.f;             // this half's running sum of P
     bool ok = true;
-    for (int u = 0; u < nsub; ++u) {
-        const int hh = u & 1;
-        const uint32_t tS = tmem + lane_addr + col_s(t, hh);
+    for (int j = 0; j < a.n_iter; ++j) {
         // warp-uniform outcome: the tcgen05.ld/st below are warp-collective
-        if (!__all_sync(0xffffffffu, mbar_wait(&sm.s_full[t][hh], static_cast<uint32_t>((u >> 1) & 1), abort_flag,
-                                               a.timeout_ns))) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&sm.s_full[t], static_cast<uint32_t>(j & 1), abort_flag, a.timeout_ns))) {
             ok = false;
             break;
         }
@@ -320,121 +339,115 @@ __device__ void softmax_group(AttnSmem& sm, const AttnArgs& a, uint32_t tmem, in
         tmem_wait_ld_x32(s[0]);
         tmem_wait_ld_x32(s[1]);
 
-        if (hh == 0) kv = list ? __ldg(list + (u >> 1)) : (u >> 1);
-        const int valid = (kv == a.nblk - 1) ? a.N - kv * 128 - kHalf * hh : kHalf;
-        if (valid < kHalf) {
+        const int kv = list ? __ldg(list + j) : j;
+        const int valid = (kv == a.nblk - 1) ? a.N - kv * 128 - 64 * hf : 64;
+        if (valid < 64) {
 #pragma unroll
             for (int q2 = 0; q2 < 2; ++q2)
 #pragma unroll
                 for (int i = 0; i < 32; ++i)
                     if (q2 * 32 + i >= valid) s[q2][i] = __float_as_uint(-INFINITY);
         }
-        // row max: four independent chains of 3-input max
-        float pm[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        float hm;
+        float* xm = &sm.xmax[j & 1][t][0][0];
+        uint64_t* xb = &sm.xbar[j & 1][t];
+        const uint32_t xpar = static_cast<uint32_t>((j >> 1) & 1);
+        if (j == 0) {
+            // the first block fixes the reference: exchange half maxima before the exponentials
+            float pm[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-        for (int q2 = 0; q2 < 2; ++q2)
+            for (int q2 = 0; q2 < 2; ++q2)
 #pragma unroll
-            for (int i = 0; i < 32; i += 8) {
-                pm[(i >> 3) & 3] = max3(pm[(i >> 3) & 3], __uint_as_float(s[q2][i]), __uint_as_float(s[q2][i + 1]));
-                pm[(i >> 3) & 3] = max3(pm[(i >> 3) & 3], __uint_as_float(s[q2][i + 2]), __uint_as_float(s[q2][i + 3]));
-                pm[(i >> 3) & 3] = max3(pm[(i >> 3) & 3], __uint_as_float(s[q2][i + 4]), __uint_as_float(s[q2][i + 5]));
-                pm[(i >> 3) & 3] = max3(pm[(i >> 3) & 3], __uint_as_float(s[q2][i + 6]), __uint_as_float(s[q2][i + 7]));
-            }
-        const float mx = fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3]));
-        const float m_new = fmaxf(m_used, mx * c);
-        // A row whose max grew by more than 2^8 rescales: P uses the new max and
-        // O is multiplied by alpha once PV of the previous half-step is done.
-        float alpha = 1.0f;
-        bool rescale_warp = false;
-        if (u == 0) {
-            m_used = m_new;
-        } else {
-            const bool need = m_new - m_used > 8.0f;
-            rescale_warp = __any_sync(0xffffffffu, need);
-            if (need) {
-                alpha = ex2_approx(m_used - m_new);
-                m_used = m_new;
-            }
-        }
-        const uint64_t negm2 = f2(-m_used, -m_used);
-        uint64_t ps = f2(0.f, 0.f);
-        // P over the first 32 columns of this S buffer: keys 32q2..32q2+31 -> columns 16q2..16q2+15
-#pragma unroll
-        for (int q2 = 0; q2 < 2; ++q2) {
-            uint32_t pk[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const uint64_t x = f2_fma(f2(__uint_as_float(s[q2][2 * i]), __uint_as_float(s[q2][2 * i + 1])), c2, negm2);
-                uint64_t pp;
-                if ((kPolyPairs >> (i & 7)) & 1u) {
-                    pp = exp2_poly_pair(x);
-                } else {
-                    float x0, x1;
-                    f2_split(x, x0, x1);
-                    pp = f2(ex2_approx(x0), ex2_approx(x1));
-                }
-                ps = f2_add(ps, pp);
-                float p0, p1;
-                f2_split(pp, p0, p1);
-                pk[i] = pack_bf16x2(p0, p1);
-            }
-            tmem_st_x16(tS + 16 * q2, pk);
-        }
-        if (rescale_warp) {
-            float l0, l1;
-            f2_split(l2, l0, l1);
-            l2 = f2(l0 * alpha, l1 * alpha);
-            // O_t must hold PV(u-1) before it is rescaled
-            if (!__all_sync(0xffffffffu, mbar_wait(&sm.pv_done[t], static_cast<uint32_t>((u - 1) & 1), abort_flag,
-                                                   a.timeout_ns))) {
+                for (int i = 0; i < 32; ++i) pm[i & 3] = fmaxf(pm[i & 3], __uint_as_float(s[q2][i]));
+            hm = fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3]));
+            xm[hf * 128 + row] = hm;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(xb);
+            if (!__all_sync(0xffffffffu, mbar_wait(xb, xpar, abort_flag, a.timeout_ns))) {
                 ok = false;
                 break;
             }
-            tc_fence_after_sync();
-#pragma unroll
-            for (int q3 = 0; q3 < 3; ++q3) {
-                uint32_t o[32];
-                tmem_ld_x32(tO + 32 * q3, o);
+            m_used = c * fmaxf(hm, xm[(hf ^ 1) * 128 + row]);
+            l += exp_store_half(s, c, m_used, tS, nullptr);
+        } else {
+            // later blocks start with the running reference (stale by design) and
+            // check the block max afterwards; only a row whose max grew by more than
+            // 2^8 recomputes its P and rescales O and its sum -- the final division
+            // by the row sum keeps the result exact either way
+            const float ps = exp_store_half(s, c, m_used, tS, &hm);
+            xm[hf * 128 + row] = hm;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(xb);
+            if (!__all_sync(0xffffffffu, mbar_wait(xb, xpar, abort_flag, a.timeout_ns))) {
+                ok = false;
+                break;
+            }
+            const float mx = c * fmaxf(hm, xm[(hf ^ 1) * 128 + row]);
+            const bool need = mx - m_used > 8.0f;
+            if (__any_sync(0xffffffffu, need)) {
+                // O_t is stable here: the commit behind s_full covers PV(j-1)
+                float alpha = 1.0f;
+                if (need) {
+                    alpha = ex2_approx(m_used - mx);
+                    m_used = mx;
+                }
+                l = l * alpha + exp_store_half(s, c, m_used, tS, nullptr);
+                uint32_t o[32], o2[16];
+                tmem_ld_x32(tO, o);
+                tmem_ld_x16(tO + 32, o2);
                 tmem_wait_ld_x32(o);
+                tmem_wait_ld_x16(o2);
 #pragma unroll
                 for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-                tmem_st_x32(tO + 32 * q3, o);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) o2[i] = __float_as_uint(__uint_as_float(o2[i]) * alpha);
+                tmem_st_x32(tO, o);
+                tmem_st_x16(tO + 32, o2);
+            } else {
+                l += ps;
             }
         }
-        l2 = f2_add(l2, ps);
+        // one arrival per warp: every lane's TMEM stores are complete and
+        // fenced before the warp converges and lane 0 releases the barrier
         tmem_wait_st();
         tc_fence_before_sync();
-        mbar_arrive(&sm.p_full[t][hh]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.p_full[t]);
     }
     if (!ok) {
         raise_timeout(a, abort_flag);
         return;
     }
-    if (!__all_sync(0xffffffffu, mbar_wait(&sm.o_done[t], 0u, abort_flag, a.timeout_ns))) {
+    // row sum = both halves
+    sm.lsum[t][hf][row] = l;
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&sm.lbar[t]);
+    if (!__all_sync(0xffffffffu, mbar_wait(&sm.lbar[t], 0u, abort_flag, a.timeout_ns)) ||
+        !__all_sync(0xffffffffu, mbar_wait(&sm.o_done[t], 0u, abort_flag, a.timeout_ns))) {
         raise_timeout(a, abort_flag);
         return;
     }
     tc_fence_after_sync();
-    float l0, l1;
-    f2_split(l2, l0, l1);
-    const float inv_l = 1.0f / (l0 + l1);
+    const float inv_l = 1.0f / (l + sm.lsum[t][hf ^ 1][row]);
     const int n = qb * 128 + row;
-    __nv_bfloat16* dst = a.o + static_cast<int64_t>(b) * a.sb + static_cast<int64_t>(n) * a.sn +
-                         static_cast<int64_t>(h) * a.sh;
+    uint32_t o[32], o2[16];
+    tmem_ld_x32(tO, o);
+    tmem_ld_x16(tO + 32, o2);
+    tmem_wait_ld_x32(o);
+    tmem_wait_ld_x16(o2);
+    if (n < a.N) {
+        __nv_bfloat16* dst = a.o + static_cast<int64_t>(b) * a.sb + static_cast<int64_t>(n) * a.sn +
+                             static_cast<int64_t>(h) * a.sh + 48 * hf;
+        uint32_t w[24];
 #pragma unroll
-    for (int q3 = 0; q3 < 3; ++q3) {
-        uint32_t o[32];
-        tmem_ld_x32(tO + 32 * q3, o);
-        tmem_wait_ld_x32(o);
-        if (n < a.N) {
-            uint32_t w[16];
+        for (int i = 0; i < 16; ++i)
+            w[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
 #pragma unroll
-            for (int i = 0; i < 16; ++i)
-                w[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
-            uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * q3);
+        for (int i = 0; i < 8; ++i)
+            w[16 + i] = pack_bf16x2(__uint_as_float(o2[2 * i]) * inv_l, __uint_as_float(o2[2 * i + 1]) * inv_l);
+        uint4* d4 = reinterpret_cast<uint4*>(dst);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) d4[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
-        }
+        for (int i = 0; i < 6; ++i) d4[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
     }
 }
 
@@ -457,11 +470,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) {
         for (int t = 0; t < 2; ++t) {
             mbar_init(&sm.q_full[t], 1);
-            for (int hh = 0; hh < 2; ++hh) {
-                mbar_init(&sm.s_full[t][hh], 1);
-                mbar_init(&sm.p_full[t][hh], 128);
-            }
-            mbar_init(&sm.pv_done[t], 1);
+            mbar_init(&sm.s_full[t], 1);
+            mbar_init(&sm.p_full[t], 8);  // one arrival per softmax warp of the tile
+            mbar_init(&sm.xbar[0][t], 8);
+            mbar_init(&sm.xbar[1][t], 8);
+            mbar_init(&sm.lbar[t], 8);
             mbar_init(&sm.o_done[t], 1);
         }
         for (int s = 0; s < kStages; ++s) {
@@ -475,7 +488,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         sm.never = 0;
         fence_barrier_init();
     }
-    if (warp == 1) {
+    if (warp == kMmaWarp) {
         tmem_alloc(&sm.tmem_base, kTmemCols);
         tmem_relinquish();
     }
@@ -485,18 +498,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem = sm.tmem_base;
     volatile int* abort_flag = &sm.abort_flag;
 
-    if (warp == 0) {
+    if (warp == kProducerWarp) {
         if ((threadIdx.x & 31) == 0) producer(sm, a, &tq, &tk, &tv, b, h, qb0, has1, l0, l1, abort_flag);
-    } else if (warp == 1) {
+    } else if (warp == kMmaWarp) {
         if ((threadIdx.x & 31) == 0) mma_issuer(sm, a, tmem, has1, l0, l1, abort_flag);
-    } else if (warp >= 4 && warp < 8) {
-        softmax_group(sm, a, tmem, 0, b, h, qb0, l0, abort_flag);
-    } else if (warp >= 8 && has1) {
-        softmax_group(sm, a, tmem, 1, b, h, qb0 + 1, l1, abort_flag);
+    } else {
+        const int wg = warp >> 2;  // softmax warpgroup: tile wg / 2, column half wg % 2
+        const int t = wg >> 1, hf = wg & 1;
+        if (t == 0 || has1) softmax_group(sm, a, tmem, t, hf, b, h, qb0 + t, t ? l1 : l0, abort_flag);
     }
     tc_fence_before_sync();
     __syncthreads();
-    if (warp == 1) {
+    if (warp == kMmaWarp) {
         tc_fence_after_sync();
         tmem_dealloc(tmem, kTmemCols);
     }
