@@ -9,22 +9,27 @@
 // 2p and 2p+1, i.e. the router's query blocks -- and streams 128-row K/V tiles
 // through shared memory: every KV block for dense attention, or each tile's
 // own routed list in sparse mode (a KV tile both lists name at the same step is
-// loaded once and shared).  Warp roles (384 threads):
-//   warp 0      TMA producer: Q tiles once, then a 3-stage K ring and a 3-stage
+// loaded once and shared).  Warp roles (576 threads, 18 warps):
+//   warps 0-15  softmax: warpgroup g = warp / 4 handles query tile g / 2 and key
+//               columns [64 (g % 2), 64 (g % 2) + 64) of every 128-key block;
+//               thread r owns row r (TMEM lane r) of that half.  It reads its 64
+//               S values from TMEM, computes exp2 in fp32 (log2 domain) with the
+//               row's reference max, writes P as packed bf16 over the first 32
+//               columns of its own S half, and agrees with the other half on the
+//               row max through shared memory and a bounded mbarrier.  The
+//               reference is fixed by the first block; a later block recomputes
+//               its P and rescales O only when a row max grew by more than 2^8
+//               (the final division by the row sum keeps this exact).  At the end
+//               each half divides its 48 O columns by the row sum, rounds once to
+//               bf16 and stores them.
+//   warp 16     TMA producer: Q tiles once, then a 3-stage K ring and a 3-stage
 //               V ring (64-byte swizzled 128 x 32 chunks, 3 per 128 x 96 tile).
-//   warp 1      owns tensor memory (512 columns) and issues tcgen05.mma from one
+//   warp 17     owns tensor memory (512 columns) and issues tcgen05.mma from one
 //               thread: S_t = Q_t K^T (M=128, N=128, K=96 as 6 steps of 16) into
 //               TMEM, O_t += P_t V (M=128, N=96, K=128 as 8 steps, P read from
 //               TMEM, V as an MN-major operand).  Order per step j:
 //               PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1), so each softmax group
 //               waits only on its own tile's chain.
-//   warps 4-7   softmax of tile 0, warps 8-11 softmax of tile 1: thread r owns
-//               query row r (TMEM lane r); it reads its S row from TMEM, keeps
-//               the running max / sum in fp32 (log2 domain, exp2), writes P as
-//               packed bf16 over the first 64 columns of S, and rescales its O
-//               row in TMEM only when the max grew by more than 2^8 (the final
-//               division by the row sum keeps this exact).  At the end it divides
-//               O by the row sum, rounds once to bf16 and stores the row.
 // TMEM columns: S_0 [0,128), S_1 [128,256), O_0 [256,352), O_1 [352,448).
 // Every mbarrier wait is bounded (timeout + CTA abort flag); a timeout sets the
 // device status word instead of hanging or trapping.
