@@ -424,7 +424,7 @@ def main():
     ap.add_argument("--workload", default=WORKLOAD, help="synthetic workload (clip32k: small profiler case)")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
-    ap.add_argument("--cpu-rows", type=int, default=1024, help="query rows of the CPU-baseline sample")
+    ap.add_argument("--cpu-rows", type=int, default=4096, help="query rows of the CPU-baseline sample")
     ap.add_argument("--ref-rows", type=int, default=128, help="query rows per reference-arm step")
     args = ap.parse_args()
     if args.warmup < 3:
