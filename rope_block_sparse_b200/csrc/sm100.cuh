@@ -79,10 +79,15 @@ __device__ __forceinline__ bool mbar_try_wait_hint(uint64_t* bar, uint32_t parit
 #define H3A_WAIT_HINT_NS 0
 #endif
 
-// Slow path of the bounded wait: polls until the phase of parity `parity`
-// completes, the CTA-wide abort flag is raised, or `limit_ns` elapses.
-static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                            uint64_t limit_ns) {
+// Bounded wait: true once the phase of parity `parity` completed; false when
+// the CTA-wide abort flag is raised or `limit_ns` elapses (the caller then
+// raises the abort flag and leaves its loop).  Fully inlined: an out-of-line
+// slow path costs a call with register saves on every wait that is not
+// already satisfied, and those waits sit on the attention kernel's critical
+// path.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                          uint64_t limit_ns) {
+    if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     for (uint32_t i = 1;; ++i) {
         if (H3A_WAIT_HINT_NS > 0 ? mbar_try_wait_hint(bar, parity, H3A_WAIT_HINT_NS) : mbar_try_wait(bar, parity))
@@ -92,14 +97,6 @@ static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parit
             if (global_timer_ns() - t0 > limit_ns) return false;
         }
     }
-}
-
-// Bounded wait: true once the phase completed; false on timeout or abort (the
-// caller then raises the abort flag and leaves its loop).
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                          uint64_t limit_ns) {
-    if (mbar_try_wait(bar, parity)) return true;
-    return mbar_wait_slow(bar, parity, abort_flag, limit_ns);
 }
 
 // ---------------------------------------------------------------- TMA
@@ -237,6 +234,8 @@ __device__ __forceinline__ void tmem_wait_ld_x16(uint32_t (&r)[16]) {
 __device__ __forceinline__ void tmem_wait_ld_x32(uint32_t (&r)[32]) {
     asm volatile("tcgen05.wait::ld.sync.aligned;" : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31]) : : "memory");
 }
+
+// 8-column variants (thread i: columns [col, col+8) of lane lane_base + i).
 
 __device__ __forceinline__ float ex2_approx(float x) {
     float y;
