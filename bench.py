@@ -165,8 +165,15 @@ def load_traffic():
         rec = json.load(f)
     out = {}
     for kernel, ent in rec.items():
-        src = os.path.join(ROOT, ent["source"])
-        if os.path.exists(src) and hashlib.sha256(open(src, "rb").read()).hexdigest() == ent["sha256"]:
+        # every file the kernel is compiled from, hashed in the listed order
+        paths = [os.path.join(ROOT, p) for p in ent["sources"]]
+        if not all(os.path.exists(p) for p in paths):
+            continue
+        h = hashlib.sha256()
+        for p in paths:
+            with open(p, "rb") as f:
+                h.update(f.read())
+        if h.hexdigest() == ent["sha256"]:
             out[kernel] = ent
     return out
 
