@@ -2,8 +2,9 @@
 
 One step = the whole hot path over one batch of the 5 s 1344x768 clip latent
 (31x48x84 = 124,992 tokens, 56 heads x 96, bf16, structured synthetic data):
-    fused QK-RMSNorm + 3D RoPE  ->  blockwise router (sparsity 0.75)
-    ->  block-sparse attention  ->  dense attention
+    fused QK-RMSNorm + 3D RoPE, with the router's block pooling folded in
+    ->  router scores and top-k (sparsity 0.75)  ->  block-sparse attention
+    ->  dense attention
 The headline value is attention TFLOP/s over the whole step (algorithmic
 FLOPs of both attention passes / step time).  Per-kernel times come from CUDA
 events on the launching stream inside the timed region.
@@ -64,8 +65,13 @@ def prologue_bytes(N: int, heads: int, B: int, d: int = 96) -> float:
 
 
 def router_bytes(N: int, heads: int, B: int, d: int = 96) -> float:
-    """The pooling pass reads Q and K once."""
+    """The separate pooling pass reads Q and K once."""
     return 2.0 * 2 * B * N * heads * d
+
+
+def pooled_bytes(N: int, heads: int, B: int, d: int = 96, block: int = 128) -> float:
+    """fp32 block means of Q and K written by the fused prologue."""
+    return 2.0 * 4 * B * heads * ((N + block - 1) // block) * d
 
 
 class ClockSampler:
@@ -198,13 +204,15 @@ def run_gpu(args, rank, world, local):
     ws = torch.empty(h3a.route_workspace_size(q), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
+    # one step: the prologue with the router's pooling folded in, the router's
+    # scores and top-k from those means, sparse attention, dense attention
     def step(ev=None):
         if ev is not None:
             ev[0].record(stream)
-        h3a.qk_norm_rope(q, k, gq, gk, grid, out=(qn, kn))
+        h3a.qk_norm_rope_pool(q, k, gq, gk, grid, workspace=ws, out=(qn, kn))
         if ev is not None:
             ev[1].record(stream)
-        h3a.route(qn, kn, SPARSITY, workspace=ws, out=blocks)
+        h3a.route_pooled(qn, SPARSITY, ws, out=blocks)
         if ev is not None:
             ev[2].record(stream)
         h3a.attention(qn, kn, v, blocks, out=o_sparse)
@@ -236,7 +244,24 @@ def run_gpu(args, rank, world, local):
     step_ms_local = float(sum(evs[i][0].elapsed_time(evs[i][4]) for i in range(args.steps)) / args.steps)
     step_ms = allreduce_max(step_ms_local, world)
     kern_ms = {name: allreduce_max(float(per[:, j].mean()), world)
-               for j, name in enumerate(["prologue", "router", "attention_sparse", "attention_dense"])}
+               for j, name in enumerate(["prologue_pool", "router_scores", "attention_sparse", "attention_dense"])}
+
+    # for comparison, outside the timed region: the separate prologue and the
+    # router with its own pooling pass
+    sep = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(5)]
+    for i in range(6):
+        e = sep[i - 1] if i > 0 else None
+        if e is not None:
+            e[0].record(stream)
+        h3a.qk_norm_rope(q, k, gq, gk, grid, out=(qn, kn))
+        if e is not None:
+            e[1].record(stream)
+        h3a.route(qn, kn, SPARSITY, workspace=ws, out=blocks)
+        if e is not None:
+            e[2].record(stream)
+    torch.cuda.synchronize()
+    kern_ms["prologue"] = allreduce_max(float(np.mean([e[0].elapsed_time(e[1]) for e in sep])), world)
+    kern_ms["router"] = allreduce_max(float(np.mean([e[1].elapsed_time(e[2]) for e in sep])), world)
 
     # end to end through the public API with host buffers
     e2e = None
@@ -278,6 +303,9 @@ def run_gpu(args, rank, world, local):
     sparse_tflops = flops_sparse / (kern_ms["attention_sparse"] * 1e-3) / 1e12
     pro_gbs = prologue_bytes(N, heads, B) / (kern_ms["prologue"] * 1e-3) / 1e9
     router_gbs = router_bytes(N, heads, B) / (kern_ms["router"] * 1e-3) / 1e9
+    fused_gbs = (prologue_bytes(N, heads, B) + pooled_bytes(N, heads, B)) / (kern_ms["prologue_pool"] * 1e-3) / 1e9
+    # the sparse path's routing cost: scores + top-k, plus what pooling adds to the prologue
+    route_cost = kern_ms["router_scores"] + max(0.0, kern_ms["prologue_pool"] - kern_ms["prologue"])
     traffic = load_traffic()
     peak_t = pk["bf16_tflops_sustained"]
     line = {
@@ -295,7 +323,8 @@ def run_gpu(args, rank, world, local):
         "data": "synthetic",
         "config": {
             "workload": f"{w.name}: B={B}, {heads} heads x 96, grid {grid[0]}x{grid[1]}x{grid[2]} = {N:,} tokens "
-                        f"per GPU; prologue + router (sparsity {SPARSITY}, k={kk}/{nblk}) + sparse + dense attention",
+                        f"per GPU; prologue with block pooling + router scores/top-k (sparsity {SPARSITY}, "
+                        f"k={kk}/{nblk}) + sparse + dense attention",
             "tokens": N, "heads": heads, "head_dim": 96, "batch_per_gpu": B, "sparsity": SPARSITY,
             "parallelism": f"dp{world} (independent clips per GPU)",
             "l2": f"inputs larger than L2 (Q, K, V {B * N * heads * 96 * 2 / 1e9:.2f} GB each); no explicit flush",
@@ -314,20 +343,26 @@ def run_gpu(args, rank, world, local):
             "algorithmic_flops_per_launch": flops_dense,
         },
         "kernels": {
-            "prologue": {"ms": round(kern_ms["prologue"], 4), "GB/s": round(pro_gbs, 1),
-                         "frac_hbm": round(pro_gbs / pk["hbm_gbs"], 4),
-                         "frac_8TBs": round(pro_gbs / 8000.0, 4),
-                         "traffic": traffic.get("prologue", {}).get("bytes_per_launch")},
-            "router": {"ms": round(kern_ms["router"], 4), "pool_read_GB/s": round(router_gbs, 1)},
+            "prologue_pool": {"ms": round(kern_ms["prologue_pool"], 4), "GB/s": round(fused_gbs, 1),
+                              "frac_hbm": round(fused_gbs / pk["hbm_gbs"], 4),
+                              "frac_8TBs": round(fused_gbs / 8000.0, 4),
+                              "traffic": traffic.get("prologue_pool", {}).get("bytes_per_launch")},
+            "router_scores": {"ms": round(kern_ms["router_scores"], 4)},
+            "separate_prologue_untimed_step": {"ms": round(kern_ms["prologue"], 4), "GB/s": round(pro_gbs, 1),
+                                               "frac_hbm": round(pro_gbs / pk["hbm_gbs"], 4),
+                                               "frac_8TBs": round(pro_gbs / 8000.0, 4),
+                                               "traffic": traffic.get("prologue", {}).get("bytes_per_launch")},
+            "separate_router_untimed_step": {"ms": round(kern_ms["router"], 4),
+                                             "pool_read_GB/s": round(router_gbs, 1)},
             "attention_sparse": {"ms": round(kern_ms["attention_sparse"], 3), "TFLOP/s": round(sparse_tflops, 2),
                                  "effective_dense_equiv_TFLOP/s":
                                      round(flops_dense / (kern_ms["attention_sparse"] * 1e-3) / 1e12, 2),
                                  "algorithmic_flops": flops_sparse},
             "attention_dense": {"ms": round(kern_ms["attention_dense"], 3), "TFLOP/s": round(dense_tflops, 2)},
             "sparse_speedup_incl_router": round(kern_ms["attention_dense"] /
-                                                (kern_ms["attention_sparse"] + kern_ms["router"]), 3),
+                                                (kern_ms["attention_sparse"] + route_cost), 3),
         },
-        "gpu_launches": args.steps * 5,
+        "gpu_launches": args.steps * 4,
         "clocks": clocks,
         "e2e": e2e,
     }

@@ -106,6 +106,36 @@ h3a_status h3a_route(const void* q, const void* k, const h3a_qkv_desc* d, double
                      int32_t block, int32_t* block_idx, int64_t* k_out, void* workspace,
                      size_t ws_bytes, h3a_stream_t stream);
 
+/* h3a_qk_norm_rope that also pools its outputs for the router, so that
+ * h3a_route_pooled can skip reading Q and K back from device memory.
+ * Source: the fused prologue of h3a_qk_norm_rope and the block pooling of
+ * h3a_route (news.cocoloop.cn MiniMax-H3 SGLang report: fused QK-RMSNorm +
+ * 3D RoPE in section "Erst drei übereinandergelegte Beschleunigungsebenen",
+ * SubBlock's blockwise router in the same section).
+ * Writes q_out / k_out exactly as h3a_qk_norm_rope does, and into workspace
+ * the fp32 means, over each 128-token block (the tail block over its real
+ * length), of the rounded outputs: the same bytes h3a_route's pooling leaves
+ * in its workspace (two fp32 [B, heads, nblk, 96] tensors, Q's first, at the
+ * offsets h3a_route uses), bit for bit.
+ * workspace : device, at least h3a_route_workspace_size(d, 128) bytes,
+ *             16-B aligned, owned by the caller; it must not overlap q, k,
+ *             q_out or k_out.
+ * Other arguments, layouts and errors: as h3a_qk_norm_rope; WORKSPACE if the
+ * workspace is null, misaligned or too small; UNSUPPORTED if B > 65535. */
+h3a_status h3a_qk_norm_rope_pool(const void* q, const void* k, const h3a_qkv_desc* d,
+                                 const float* gamma_q, const float* gamma_k, h3a_grid grid,
+                                 double theta, float eps, void* q_out, void* k_out,
+                                 void* workspace, size_t ws_bytes, h3a_stream_t stream);
+
+/* The scoring and top-k half of h3a_route, from block means that
+ * h3a_qk_norm_rope_pool left in the workspace (same source and rule as
+ * h3a_route).  d describes the Q/K tensors that were pooled; block_idx,
+ * k_out and the result are those of h3a_route on the prologue's outputs.
+ * The workspace is only read.  Errors: as h3a_route. */
+h3a_status h3a_route_pooled(const h3a_qkv_desc* d, double sparsity, int32_t block,
+                            int32_t* block_idx, int64_t* k_out, const void* workspace,
+                            size_t ws_bytes, h3a_stream_t stream);
+
 /* Capacity of the scratch built into h3a_route_noalloc: 64 MiB, enough for
  * B * heads * ceil(N / 128) <= 87,381 (e.g. 56 heads of a 124,992-token clip). */
 #define H3A_ROUTE_NOALLOC_MAX_BYTES ((size_t)64 << 20)

@@ -113,6 +113,43 @@ cudaError_t make_qkv_tensor_map(CUtensorMap* map, const void* base, const Shape&
 
 using namespace h3a;
 
+namespace {
+
+// Shared checks of the router's shape, sparsity and workspace; on success
+// fills nblk, k and the two pooled halves of the workspace.
+h3a_status route_setup(const Shape& s, double sparsity, int32_t block, const void* workspace, size_t ws_bytes,
+                       int* nblk, int64_t* kk, float** pq, float** pk) {
+    if (block != kBlock) return H3A_ERR_UNSUPPORTED;
+    if (!(sparsity >= 0.0 && sparsity < 1.0)) return H3A_ERR_INVALID_ARG;
+    *nblk = (s.N + kBlock - 1) / kBlock;
+    if (*nblk > route_max_blocks()) return H3A_ERR_UNSUPPORTED;
+    if (static_cast<int64_t>(s.B) * s.heads > 65535) return H3A_ERR_UNSUPPORTED;
+    const size_t half = pooled_bytes(s, *nblk);
+    if (workspace == nullptr || !aligned16(workspace) || ws_bytes < 2 * half) return H3A_ERR_WORKSPACE;
+    *kk = h3a_route_k(*nblk, sparsity);
+    *pq = static_cast<float*>(const_cast<void*>(workspace));
+    *pk = reinterpret_cast<float*>(static_cast<char*>(const_cast<void*>(workspace)) + half);
+    return H3A_OK;
+}
+
+// Shared checks of the prologue's arguments.
+h3a_status prologue_check(const void* q, const void* k, const h3a_qkv_desc* d, const float* gamma_q,
+                          const float* gamma_k, h3a_grid grid, double theta, float eps, const void* q_out,
+                          const void* k_out, Shape* s) {
+    h3a_status rc = check_desc(d, s);
+    if (rc != H3A_OK) return rc;
+    if (!q || !k || !gamma_q || !gamma_k || !q_out || !k_out) return H3A_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(q_out) || !aligned16(k_out)) return H3A_ERR_INVALID_ARG;
+    if (!(reinterpret_cast<uintptr_t>(gamma_q) % 4 == 0 && reinterpret_cast<uintptr_t>(gamma_k) % 4 == 0))
+        return H3A_ERR_INVALID_ARG;
+    if (grid.T < 1 || grid.H < 1 || grid.W < 1) return H3A_ERR_INVALID_ARG;
+    if (static_cast<int64_t>(grid.T) * grid.H * grid.W != d->N) return H3A_ERR_INVALID_ARG;
+    if (!(eps >= 0.0f) || !(theta > 0.0)) return H3A_ERR_INVALID_ARG;
+    return H3A_OK;
+}
+
+}  // namespace
+
 extern "C" {
 
 const char* h3a_status_string(h3a_status s) {
@@ -133,15 +170,8 @@ h3a_status h3a_qk_norm_rope(const void* q, const void* k, const h3a_qkv_desc* d,
                             const float* gamma_k, h3a_grid grid, double theta, float eps, void* q_out, void* k_out,
                             h3a_stream_t stream) {
     Shape s;
-    h3a_status rc = check_desc(d, &s);
+    h3a_status rc = prologue_check(q, k, d, gamma_q, gamma_k, grid, theta, eps, q_out, k_out, &s);
     if (rc != H3A_OK) return rc;
-    if (!q || !k || !gamma_q || !gamma_k || !q_out || !k_out) return H3A_ERR_INVALID_ARG;
-    if (!aligned16(q) || !aligned16(k) || !aligned16(q_out) || !aligned16(k_out)) return H3A_ERR_INVALID_ARG;
-    if (!(reinterpret_cast<uintptr_t>(gamma_q) % 4 == 0 && reinterpret_cast<uintptr_t>(gamma_k) % 4 == 0))
-        return H3A_ERR_INVALID_ARG;
-    if (grid.T < 1 || grid.H < 1 || grid.W < 1) return H3A_ERR_INVALID_ARG;
-    if (static_cast<int64_t>(grid.T) * grid.H * grid.W != d->N) return H3A_ERR_INVALID_ARG;
-    if (!(eps >= 0.0f) || !(theta > 0.0)) return H3A_ERR_INVALID_ARG;
     cudaError_t e = launch_qk_norm_rope(q, k, q_out, k_out, gamma_q, gamma_k, s, grid.T, grid.H, grid.W, theta, eps,
                                         reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? H3A_OK : cuda_fail(e);
@@ -174,18 +204,48 @@ h3a_status h3a_route(const void* q, const void* k, const h3a_qkv_desc* d, double
     if (block != kBlock) return H3A_ERR_UNSUPPORTED;
     if (!q || !k || !block_idx) return H3A_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || (reinterpret_cast<uintptr_t>(block_idx) & 3u)) return H3A_ERR_INVALID_ARG;
-    if (!(sparsity >= 0.0 && sparsity < 1.0)) return H3A_ERR_INVALID_ARG;
-    const int nblk = (s.N + kBlock - 1) / kBlock;
-    if (nblk > route_max_blocks()) return H3A_ERR_UNSUPPORTED;
-    if (static_cast<int64_t>(s.B) * s.heads > 65535) return H3A_ERR_UNSUPPORTED;
-    const size_t half = pooled_bytes(s, nblk);
-    if (workspace == nullptr || !aligned16(workspace) || ws_bytes < 2 * half) return H3A_ERR_WORKSPACE;
-    const int64_t kk = h3a_route_k(nblk, sparsity);
+    int nblk;
+    int64_t kk;
+    float *pq, *pk;
+    rc = route_setup(s, sparsity, block, workspace, ws_bytes, &nblk, &kk, &pq, &pk);
+    if (rc != H3A_OK) return rc;
     if (k_out) *k_out = kk;
-    float* pq = static_cast<float*>(workspace);
-    float* pk = reinterpret_cast<float*>(static_cast<char*>(workspace) + half);
     cudaError_t e = launch_route(q, k, s, nblk, static_cast<int>(kk), pq, pk, block_idx,
                                  reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? H3A_OK : cuda_fail(e);
+}
+
+h3a_status h3a_qk_norm_rope_pool(const void* q, const void* k, const h3a_qkv_desc* d, const float* gamma_q,
+                                 const float* gamma_k, h3a_grid grid, double theta, float eps, void* q_out,
+                                 void* k_out, void* workspace, size_t ws_bytes, h3a_stream_t stream) {
+    Shape s;
+    h3a_status rc = prologue_check(q, k, d, gamma_q, gamma_k, grid, theta, eps, q_out, k_out, &s);
+    if (rc != H3A_OK) return rc;
+    const int nblk = (s.N + kBlock - 1) / kBlock;
+    if (s.B > 65535 || (s.heads + 27) / 28 > 65535) return H3A_ERR_UNSUPPORTED;
+    const size_t half = pooled_bytes(s, nblk);
+    if (workspace == nullptr || !aligned16(workspace) || ws_bytes < 2 * half) return H3A_ERR_WORKSPACE;
+    float* pq = static_cast<float*>(workspace);
+    float* pk = reinterpret_cast<float*>(static_cast<char*>(workspace) + half);
+    cudaError_t e = launch_qk_norm_rope_pool(q, k, q_out, k_out, gamma_q, gamma_k, s, grid.H, grid.W, theta, eps, pq,
+                                             pk, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? H3A_OK : cuda_fail(e);
+}
+
+h3a_status h3a_route_pooled(const h3a_qkv_desc* d, double sparsity, int32_t block, int32_t* block_idx,
+                            int64_t* k_out, const void* workspace, size_t ws_bytes, h3a_stream_t stream) {
+    Shape s;
+    h3a_status rc = check_desc(d, &s);
+    if (rc != H3A_OK) return rc;
+    if (!block_idx || (reinterpret_cast<uintptr_t>(block_idx) & 3u)) return H3A_ERR_INVALID_ARG;
+    int nblk;
+    int64_t kk;
+    float *pq, *pk;
+    rc = route_setup(s, sparsity, block, workspace, ws_bytes, &nblk, &kk, &pq, &pk);
+    if (rc != H3A_OK) return rc;
+    if (k_out) *k_out = kk;
+    cudaError_t e = launch_route_scores(pq, pk, s, nblk, static_cast<int>(kk), block_idx,
+                                        reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? H3A_OK : cuda_fail(e);
 }
 

@@ -24,10 +24,19 @@ cudaError_t launch_qk_norm_rope(const void* q, const void* k, void* q_out, void*
                                 const float* gamma_k, const Shape& s, int T, int H, int W, double theta,
                                 float eps, cudaStream_t st);
 
+// Prologue that also writes the fp32 means of its rounded outputs over
+// 128-token blocks into pool_q / pool_k ([B, heads, nblk, 96]) (prologue.cu).
+cudaError_t launch_qk_norm_rope_pool(const void* q, const void* k, void* q_out, void* k_out, const float* gamma_q,
+                                     const float* gamma_k, const Shape& s, int H, int W, double theta, float eps,
+                                     float* pool_q, float* pool_k, cudaStream_t st);
+
 // Router (router.cu): block means of q and k into pooled_q / pooled_k
 // ([B, heads, nblk, 96] fp32), then scores and top-k into idx.
 cudaError_t launch_route(const void* q, const void* k, const Shape& s, int nblk, int kk, float* pooled_q,
                          float* pooled_k, int32_t* idx, cudaStream_t st);
+// Scores and top-k only, from block means already in pooled_q / pooled_k.
+cudaError_t launch_route_scores(const float* pooled_q, const float* pooled_k, const Shape& s, int nblk, int kk,
+                                int32_t* idx, cudaStream_t st);
 // Largest nblk the score/top-k kernel supports (shared-memory bound).
 int route_max_blocks();
 

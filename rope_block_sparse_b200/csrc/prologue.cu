@@ -1,7 +1,8 @@
 // Fused QK-RMSNorm + 3D RoPE prologue (news.cocoloop.cn MiniMax-H3 SGLang
 // report, fused-operator paragraph: QK-RMSNorm with 3D RoPE in one kernel, no
 // change to the result; 3D multimodal RoPE from the 52hbtv.com H3-Image page,
-// section 二, model table).
+// section 二, model table), and the same prologue with the router's block
+// pooling folded in (qk_norm_rope_pool_kernel, at the end of this file).
 //
 // HBM-bound: every element of Q and K is read once and written once (4 bytes
 // per element, 43,008 bytes per token at 56 heads).  One warp owns one token at
@@ -40,6 +41,10 @@ struct PrologueArgs {
     // theta^(-2j/32) as an unevaluated sum hi + lo of two floats
     float freq_hi[kPairsPerSection];
     float freq_lo[kPairsPerSection];
+    // block pooling (qk_norm_rope_pool_kernel only): fp32 [B, heads, nblk, 96]
+    float* pool_q;
+    float* pool_k;
+    int nblk;
 };
 
 __device__ __forceinline__ void unpack4(uint2 v, float* x) {
@@ -54,10 +59,12 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
     return *reinterpret_cast<uint32_t*>(&h);
 }
 
-// Normalise, scale, rotate and store one lane's 12 channels of one head.
-__device__ __forceinline__ void norm_rope_store(const uint2 (&raw)[3], const float (&g)[kChanPerLane],
-                                                const float (&cs)[kPairsPerLane], const float (&sn)[kPairsPerLane],
-                                                float eps, bool active, __nv_bfloat16* dst) {
+// Normalise, scale and rotate one lane's 12 channels of one head; out[p] holds
+// the rounded pair p as packed bf16.  Every lane of the warp must take part
+// (the RMS sum is reduced across each 8-lane group).
+__device__ __forceinline__ void norm_rope(const uint2 (&raw)[3], const float (&g)[kChanPerLane],
+                                          const float (&cs)[kPairsPerLane], const float (&sn)[kPairsPerLane],
+                                          float eps, uint32_t (&out)[kPairsPerLane]) {
     float x[kChanPerLane];
     unpack4(raw[0], x);
     unpack4(raw[1], x + 4);
@@ -69,7 +76,6 @@ __device__ __forceinline__ void norm_rope_store(const uint2 (&raw)[3], const flo
     ss += __shfl_xor_sync(0xffffffffu, ss, 2);
     ss += __shfl_xor_sync(0xffffffffu, ss, 4);
     const float r = rsqrtf(ss * (1.0f / kHeadDim) + eps);
-    uint32_t out[kPairsPerLane];
 #pragma unroll
     for (int p = 0; p < kPairsPerLane; ++p) {
         const float y0 = x[2 * p] * r * g[2 * p];
@@ -78,12 +84,42 @@ __device__ __forceinline__ void norm_rope_store(const uint2 (&raw)[3], const flo
         const float z1 = y0 * sn[p] + y1 * cs[p];
         out[p] = pack2(z0, z1);
     }
+}
+
+__device__ __forceinline__ void store3(const uint32_t (&out)[kPairsPerLane], bool active, __nv_bfloat16* dst) {
     if (active) {
         uint2* d = reinterpret_cast<uint2*>(dst);
         d[0] = make_uint2(out[0], out[1]);
         d[1] = make_uint2(out[2], out[3]);
         d[2] = make_uint2(out[4], out[5]);
     }
+}
+
+__device__ __forceinline__ void norm_rope_store(const uint2 (&raw)[3], const float (&g)[kChanPerLane],
+                                                const float (&cs)[kPairsPerLane], const float (&sn)[kPairsPerLane],
+                                                float eps, bool active, __nv_bfloat16* dst) {
+    uint32_t out[kPairsPerLane];
+    norm_rope(raw, g, cs, sn, eps, out);
+    store3(out, active, dst);
+}
+
+// cos / sin of the rotation of pair `pair` (0..47 within a head: section
+// pair / 16, index j = pair % 16) at grid position pos: fp32 sincos of the high
+// part of the angle pos * theta^(-2j/32), corrected to first order by its low
+// part (the frequency is an unevaluated sum hi + lo of two floats).
+__device__ __forceinline__ void rotation(int pt, int ph, int pw, int pair, const float* freq_hi,
+                                         const float* freq_lo, float& c_out, float& s_out) {
+    const int axis = pair / kPairsPerSection;
+    const int j = pair % kPairsPerSection;
+    // selects, not an indexed array: axis depends on the lane
+    const float ps = static_cast<float>(axis == 0 ? pt : (axis == 1 ? ph : pw));
+    const float hi = freq_hi[j];
+    const float a_hi = ps * hi;
+    const float a_lo = fmaf(ps, hi, -a_hi) + ps * freq_lo[j];
+    float s, c;
+    sincosf(a_hi, &s, &c);
+    c_out = fmaf(-a_lo, s, c);
+    s_out = fmaf(a_lo, c, s);
 }
 
 __device__ __forceinline__ void load3(const __nv_bfloat16* src, bool active, uint2 (&raw)[3]) {
@@ -116,24 +152,13 @@ __global__ void __launch_bounds__(kThreads, 3) qk_norm_rope_kernel(const Prologu
          tok += warps) {
         const int b = static_cast<int>(tok / a.N);
         const int n = static_cast<int>(tok - static_cast<int64_t>(b) * a.N);
-        const int pos[3] = {n / (a.H * a.W), (n / a.W) % a.H, n % a.W};
+        const int pt = n / (a.H * a.W), ph = (n / a.W) % a.H, pw = n % a.W;
 
         // rotation of this lane's six pairs at this token
         float cs[kPairsPerLane], sn[kPairsPerLane];
 #pragma unroll
-        for (int p = 0; p < kPairsPerLane; ++p) {
-            const int pair = sub * kPairsPerLane + p;  // 0..47 within the head
-            const int axis = pair / kPairsPerSection;
-            const int j = pair % kPairsPerSection;
-            const float ps = static_cast<float>(pos[axis]);
-            const float hi = a.freq_hi[j];
-            const float a_hi = ps * hi;
-            const float a_lo = fmaf(ps, hi, -a_hi) + ps * a.freq_lo[j];
-            float s, c;
-            sincosf(a_hi, &s, &c);
-            cs[p] = fmaf(-a_lo, s, c);
-            sn[p] = fmaf(a_lo, c, s);
-        }
+        for (int p = 0; p < kPairsPerLane; ++p)
+            rotation(pt, ph, pw, sub * kPairsPerLane + p, a.freq_hi, a.freq_lo, cs[p], sn[p]);
 
         const int64_t tok_off = static_cast<int64_t>(b) * a.sb + static_cast<int64_t>(n) * a.sn + c0;
         for (int hg = 0; hg < head_groups; hg += 2) {
@@ -151,6 +176,131 @@ __global__ void __launch_bounds__(kThreads, 3) qk_norm_rope_kernel(const Prologu
             norm_rope_store(rq1, gq, cs, sn, a.eps, act1, a.qo + off1);
             norm_rope_store(rk1, gk, cs, sn, a.eps, act1, a.ko + off1);
         }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Prologue + block pooling.  The router pools the prologue's outputs over
+// 128-token blocks (news.cocoloop.cn MiniMax-H3 SGLang report, SubBlock
+// paragraph; block means as fixed by the problem statement); this kernel
+// produces those means while the rounded outputs are still in registers, so
+// the router need not read Q and K back from HBM.
+//
+// One CTA per (batch, 128-token block, chunk of 28 heads); warp w owns heads
+// 28*chunk + 4w .. +3 with the prologue's lane layout (8 lanes per head, 12
+// channels per lane) and walks the block's tokens in order.  Each (head,
+// channel) sum therefore lives in one lane and adds the bf16-rounded outputs
+// in token order, exactly as the separate pooling kernel does, so the means
+// are bit-identical to it.  The rotation of every (token, pair) of the block
+// is computed once per CTA into shared memory: a warp now covers 4 heads per
+// token instead of 56, and computing the rotation per warp would cost more
+// issue slots than the HBM-bound prologue has to spare.  Each warp keeps the
+// loads of four tokens in flight (128 registers, two CTAs per SM): with one
+// token per iteration the kernel reached only a third of HBM bandwidth.
+constexpr int kPoolWarps = 7;
+constexpr int kPoolThreads = 32 * kPoolWarps;              // 224
+constexpr int kPoolHeadsPerCta = 4 * kPoolWarps;           // 28
+constexpr int kPairsPerHead = kHeadDim / 2;                // 48
+constexpr size_t kPoolSmemBytes = sizeof(float2) * kBlock * kPairsPerHead;  // 48 KB
+#ifndef H3A_POOL_UNROLL
+#define H3A_POOL_UNROLL 4
+#endif
+constexpr int kPoolUnroll = H3A_POOL_UNROLL;  // tokens whose loads are in flight together
+
+__device__ __forceinline__ void add_rounded(const uint32_t (&out)[kPairsPerLane], float (&acc)[kChanPerLane]) {
+#pragma unroll
+    for (int p = 0; p < kPairsPerLane; ++p) {
+        acc[2 * p] += __uint_as_float(out[p] << 16);
+        acc[2 * p + 1] += __uint_as_float(out[p] & 0xFFFF0000u);
+    }
+}
+
+__global__ void __launch_bounds__(kPoolThreads, 2) qk_norm_rope_pool_kernel(const PrologueArgs a) {
+    extern __shared__ float2 rot[];  // [kBlock][kPairsPerHead]: (cos, sin)
+    const int blk = blockIdx.x, b = blockIdx.y, chunk = blockIdx.z;
+    const int n0 = blk * kBlock;
+    const int len = min(a.N - n0, kBlock);
+
+    for (int e = threadIdx.x; e < len * kPairsPerHead; e += kPoolThreads) {
+        const int i = e / kPairsPerHead, pair = e - i * kPairsPerHead;
+        const int n = n0 + i;
+        float c, sn;
+        rotation(n / (a.H * a.W), (n / a.W) % a.H, n % a.W, pair, a.freq_hi, a.freq_lo, c, sn);
+        rot[e] = make_float2(c, sn);
+    }
+    __syncthreads();
+
+    const int lane = threadIdx.x & 31;
+    const int sub = lane & 7;
+    const int c0 = sub * kChanPerLane;
+    const int h = chunk * kPoolHeadsPerCta + (threadIdx.x >> 5) * 4 + (lane >> 3);
+    const bool active = h < a.heads;
+    float gq[kChanPerLane], gk[kChanPerLane];
+#pragma unroll
+    for (int i = 0; i < kChanPerLane; ++i) {
+        gq[i] = __ldg(a.gq + c0 + i);
+        gk[i] = __ldg(a.gk + c0 + i);
+    }
+    float accq[kChanPerLane], acck[kChanPerLane];
+#pragma unroll
+    for (int i = 0; i < kChanPerLane; ++i) accq[i] = acck[i] = 0.f;
+
+    const int64_t base = static_cast<int64_t>(b) * a.sb + static_cast<int64_t>(h) * a.sh + c0;
+    // kPoolUnroll tokens per iteration, all their loads issued first; the
+    // sums still add the tokens in order
+    for (int i = 0; i < len; i += kPoolUnroll) {
+        uint2 rq[kPoolUnroll][3], rk[kPoolUnroll][3];
+#pragma unroll
+        for (int u = 0; u < kPoolUnroll; ++u) {
+            const int64_t off = base + static_cast<int64_t>(n0 + i + u) * a.sn;
+            const bool act = active && i + u < len;
+            load3(a.q + off, act, rq[u]);
+            load3(a.k + off, act, rk[u]);
+        }
+#pragma unroll
+        for (int u = 0; u < kPoolUnroll; ++u) {
+            if (i + u >= len) break;
+            float cs[kPairsPerLane], sn[kPairsPerLane];
+#pragma unroll
+            for (int p = 0; p < kPairsPerLane; ++p) {
+                const float2 v = rot[(i + u) * kPairsPerHead + sub * kPairsPerLane + p];
+                cs[p] = v.x;
+                sn[p] = v.y;
+            }
+            const int64_t off = base + static_cast<int64_t>(n0 + i + u) * a.sn;
+            uint32_t oq[kPairsPerLane], ok[kPairsPerLane];
+            norm_rope(rq[u], gq, cs, sn, a.eps, oq);
+            norm_rope(rk[u], gk, cs, sn, a.eps, ok);
+            store3(oq, active, a.qo + off);
+            store3(ok, active, a.ko + off);
+            add_rounded(oq, accq);
+            add_rounded(ok, acck);
+        }
+    }
+    if (!active) return;
+    const float inv_len = 1.0f / static_cast<float>(len);
+    const int64_t dst = ((static_cast<int64_t>(b) * a.heads + h) * a.nblk + blk) * kHeadDim + c0;
+    float4* dq = reinterpret_cast<float4*>(a.pool_q + dst);
+    float4* dk = reinterpret_cast<float4*>(a.pool_k + dst);
+#pragma unroll
+    for (int u = 0; u < kChanPerLane / 4; ++u) {
+        dq[u] = make_float4(accq[4 * u] * inv_len, accq[4 * u + 1] * inv_len, accq[4 * u + 2] * inv_len,
+                            accq[4 * u + 3] * inv_len);
+        dk[u] = make_float4(acck[4 * u] * inv_len, acck[4 * u + 1] * inv_len, acck[4 * u + 2] * inv_len,
+                            acck[4 * u + 3] * inv_len);
+    }
+}
+
+}  // namespace
+
+namespace {
+
+// theta^(-2j/32), j = 0..15, split into an unevaluated sum hi + lo of two floats.
+void set_frequencies(double theta, PrologueArgs& a) {
+    for (int j = 0; j < kPairsPerSection; ++j) {
+        const double f = std::pow(theta, -2.0 * j / (kHeadDim / 3));
+        a.freq_hi[j] = static_cast<float>(f);
+        a.freq_lo[j] = static_cast<float>(f - static_cast<double>(a.freq_hi[j]));
     }
 }
 
@@ -176,11 +326,9 @@ cudaError_t launch_qk_norm_rope(const void* q, const void* k, void* q_out, void*
     a.sn = s.sn;
     a.sh = s.sh;
     a.eps = eps;
-    for (int j = 0; j < kPairsPerSection; ++j) {
-        const double f = std::pow(theta, -2.0 * j / (kHeadDim / 3));
-        a.freq_hi[j] = static_cast<float>(f);
-        a.freq_lo[j] = static_cast<float>(f - static_cast<double>(a.freq_hi[j]));
-    }
+    set_frequencies(theta, a);
+    a.pool_q = a.pool_k = nullptr;
+    a.nblk = 0;
     if (a.tokens == 0) return cudaSuccess;
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
@@ -190,6 +338,37 @@ cudaError_t launch_qk_norm_rope(const void* q, const void* k, void* q_out, void*
     const int64_t cap = static_cast<int64_t>(sms) * 3 * 8;
     if (blocks > cap) blocks = cap;
     qk_norm_rope_kernel<<<static_cast<unsigned>(blocks), kThreads, 0, st>>>(a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_qk_norm_rope_pool(const void* q, const void* k, void* q_out, void* k_out, const float* gamma_q,
+                                     const float* gamma_k, const Shape& s, int H, int W, double theta, float eps,
+                                     float* pool_q, float* pool_k, cudaStream_t st) {
+    PrologueArgs a;
+    a.q = static_cast<const __nv_bfloat16*>(q);
+    a.k = static_cast<const __nv_bfloat16*>(k);
+    a.qo = static_cast<__nv_bfloat16*>(q_out);
+    a.ko = static_cast<__nv_bfloat16*>(k_out);
+    a.gq = gamma_q;
+    a.gk = gamma_k;
+    a.tokens = static_cast<int64_t>(s.B) * s.N;
+    a.N = s.N;
+    a.heads = s.heads;
+    a.H = H;
+    a.W = W;
+    a.sb = s.sb;
+    a.sn = s.sn;
+    a.sh = s.sh;
+    a.eps = eps;
+    set_frequencies(theta, a);
+    a.pool_q = pool_q;
+    a.pool_k = pool_k;
+    a.nblk = (s.N + kBlock - 1) / kBlock;
+    const int chunks = (s.heads + kPoolHeadsPerCta - 1) / kPoolHeadsPerCta;
+    cudaError_t e = cudaFuncSetAttribute(qk_norm_rope_pool_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(kPoolSmemBytes));
+    if (e != cudaSuccess) return e;
+    qk_norm_rope_pool_kernel<<<dim3(a.nblk, s.B, chunks), kPoolThreads, kPoolSmemBytes, st>>>(a);
     return cudaGetLastError();
 }
 

@@ -250,6 +250,23 @@ int route_max_blocks() {
     return static_cast<int>((kScoreSmemLimit - score_smem_bytes(0)) / (kRowsPerCta * sizeof(float)));
 }
 
+cudaError_t launch_route_scores(const float* pooled_q, const float* pooled_k, const Shape& s, int nblk, int kk,
+                                int32_t* idx, cudaStream_t st) {
+    ScoreArgs a;
+    a.qp = pooled_q;
+    a.kp = pooled_k;
+    a.idx = idx;
+    a.nblk = nblk;
+    a.kk = kk;
+    a.inv_sqrt_d = static_cast<float>(1.0 / std::sqrt(static_cast<double>(kHeadDim)));
+    const size_t smem = score_smem_bytes(nblk);
+    cudaError_t e =
+        cudaFuncSetAttribute(score_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    score_topk_kernel<<<dim3((nblk + kRowsPerCta - 1) / kRowsPerCta, s.B * s.heads), kScoreThreads, smem, st>>>(a);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_route(const void* q, const void* k, const Shape& s, int nblk, int kk, float* pooled_q,
                          float* pooled_k, int32_t* idx, cudaStream_t st) {
     PoolArgs p;
@@ -267,19 +284,7 @@ cudaError_t launch_route(const void* q, const void* k, const Shape& s, int nblk,
     block_pool_kernel<<<dim3(nblk, s.B, 2 * chunks), kPoolThreads, 0, st>>>(p);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-
-    ScoreArgs a;
-    a.qp = pooled_q;
-    a.kp = pooled_k;
-    a.idx = idx;
-    a.nblk = nblk;
-    a.kk = kk;
-    a.inv_sqrt_d = static_cast<float>(1.0 / std::sqrt(static_cast<double>(kHeadDim)));
-    const size_t smem = score_smem_bytes(nblk);
-    e = cudaFuncSetAttribute(score_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    score_topk_kernel<<<dim3((nblk + kRowsPerCta - 1) / kRowsPerCta, s.B * s.heads), kScoreThreads, smem, st>>>(a);
-    return cudaGetLastError();
+    return launch_route_scores(pooled_q, pooled_k, s, nblk, kk, idx, st);
 }
 
 }  // namespace h3a

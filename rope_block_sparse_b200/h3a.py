@@ -25,7 +25,8 @@ STATUS_NAMES = {0: "H3A_OK", 1: "H3A_ERR_INVALID_ARG", 2: "H3A_ERR_UNSUPPORTED",
 # Every function the header declares; checked by the ABI test.
 EXPORTS = ("h3a_qk_norm_rope", "h3a_route_k", "h3a_route_workspace_size", "h3a_route", "h3a_attention",
            "h3a_status_string", "h3a_last_cuda_error_string", "h3a_last_device_error",
-           "h3a_selftest_wait_timeout", "h3a_selftest_mma", "h3a_selftest_exp2", "h3a_route_noalloc")
+           "h3a_selftest_wait_timeout", "h3a_selftest_mma", "h3a_selftest_exp2", "h3a_route_noalloc",
+           "h3a_qk_norm_rope_pool", "h3a_route_pooled")
 ROUTE_NOALLOC_MAX_BYTES = 64 << 20  # H3A_ROUTE_NOALLOC_MAX_BYTES
 
 
@@ -87,6 +88,12 @@ def load() -> ctypes.CDLL:
     lib.h3a_selftest_exp2.restype = st
     lib.h3a_route_noalloc.argtypes = [P, P, ctypes.POINTER(QkvDesc), f64, i32, P, ctypes.POINTER(ctypes.c_int64), P]
     lib.h3a_route_noalloc.restype = st
+    lib.h3a_qk_norm_rope_pool.argtypes = [P, P, ctypes.POINTER(QkvDesc), P, P, Grid, f64, f32, P, P, P,
+                                          ctypes.c_size_t, P]
+    lib.h3a_qk_norm_rope_pool.restype = st
+    lib.h3a_route_pooled.argtypes = [ctypes.POINTER(QkvDesc), f64, i32, P, ctypes.POINTER(ctypes.c_int64), P,
+                                     ctypes.c_size_t, P]
+    lib.h3a_route_pooled.restype = st
     _lib = lib
     return lib
 
@@ -126,28 +133,88 @@ def _check_qkv(*ts: torch.Tensor):
             raise ValueError("q, k, v (and outputs) must share shape and strides")
 
 
+def _prologue_outputs(q, k, gamma_q, gamma_k, inplace, out):
+    _check_qkv(q, k)
+    for g in (gamma_q, gamma_k):
+        if not g.is_cuda or g.dtype != torch.float32 or g.numel() != HEAD_DIM or not g.is_contiguous():
+            raise ValueError("gammas must be contiguous fp32 [96] CUDA tensors")
+    if inplace:
+        return q, k
+    if out is not None:
+        qo, ko = out
+        _check_qkv(q, qo, ko)
+        return qo, ko
+    return torch.empty_like(q), torch.empty_like(k)
+
+
 def qk_norm_rope(q: torch.Tensor, k: torch.Tensor, gamma_q: torch.Tensor, gamma_k: torch.Tensor, grid,
                  theta: float = 10000.0, eps: float = 1e-6, inplace: bool = False, out=None):
     """Fused QK-RMSNorm + 3D RoPE over [B, N, heads, 96] bf16 q and k; returns (q_out, k_out).
 
     inplace=True overwrites q and k; out=(q_out, k_out) writes into given tensors."""
     lib = load()
-    _check_qkv(q, k)
-    for g in (gamma_q, gamma_k):
-        if not g.is_cuda or g.dtype != torch.float32 or g.numel() != HEAD_DIM or not g.is_contiguous():
-            raise ValueError("gammas must be contiguous fp32 [96] CUDA tensors")
-    if inplace:
-        qo, ko = q, k
-    elif out is not None:
-        qo, ko = out
-        _check_qkv(q, qo, ko)
-    else:
-        qo, ko = torch.empty_like(q), torch.empty_like(k)
+    qo, ko = _prologue_outputs(q, k, gamma_q, gamma_k, inplace, out)
     d = desc_of(q)
     _check("h3a_qk_norm_rope", lib.h3a_qk_norm_rope(_ptr(q), _ptr(k), ctypes.byref(d), _ptr(gamma_q),
                                                     _ptr(gamma_k), Grid(*grid), float(theta), float(eps),
                                                     _ptr(qo), _ptr(ko), _stream_handle()))
     return qo, ko
+
+
+def _workspace(q: torch.Tensor, workspace: torch.Tensor | None, block: int = BLOCK) -> torch.Tensor:
+    need = route_workspace_size(q, block)
+    if workspace is None:
+        return torch.empty(need, dtype=torch.uint8, device=q.device)
+    if not workspace.is_cuda or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    return workspace
+
+
+def qk_norm_rope_pool(q: torch.Tensor, k: torch.Tensor, gamma_q: torch.Tensor, gamma_k: torch.Tensor, grid,
+                      theta: float = 10000.0, eps: float = 1e-6, workspace: torch.Tensor | None = None,
+                      inplace: bool = False, out=None):
+    """qk_norm_rope that also leaves the router's fp32 block means in `workspace`
+    (as route() would compute them); returns (q_out, k_out, workspace) for route_pooled()."""
+    lib = load()
+    qo, ko = _prologue_outputs(q, k, gamma_q, gamma_k, inplace, out)
+    workspace = _workspace(q, workspace)
+    d = desc_of(q)
+    _check("h3a_qk_norm_rope_pool",
+           lib.h3a_qk_norm_rope_pool(_ptr(q), _ptr(k), ctypes.byref(d), _ptr(gamma_q), _ptr(gamma_k), Grid(*grid),
+                                     float(theta), float(eps), _ptr(qo), _ptr(ko), _ptr(workspace),
+                                     workspace.numel() * workspace.element_size(), _stream_handle()))
+    return qo, ko, workspace
+
+
+def route_pooled(q: torch.Tensor, sparsity: float, workspace: torch.Tensor, block: int = BLOCK,
+                 out: torch.Tensor | None = None) -> torch.Tensor:
+    """Scores + top-k from the block means qk_norm_rope_pool left in `workspace`
+    (q only supplies the shape); same result as route() on the prologue outputs."""
+    lib = load()
+    if not q.is_cuda:
+        raise ValueError("tensors must be on a CUDA device (libh3a has no CPU path)")
+    B, N, H, _ = q.shape
+    nblk = (N + block - 1) // block
+    kk = route_k(nblk, sparsity)
+    if kk < 0:
+        raise ValueError(f"sparsity {sparsity} outside [0, 1)")
+    out = _route_out(q, nblk, kk, out)
+    k_out = ctypes.c_int64(0)
+    d = desc_of(q)
+    _check("h3a_route_pooled", lib.h3a_route_pooled(ctypes.byref(d), float(sparsity), block, _ptr(out),
+                                                    ctypes.byref(k_out), _ptr(workspace),
+                                                    workspace.numel() * workspace.element_size(),
+                                                    _stream_handle()))
+    return out
+
+
+def _route_out(q: torch.Tensor, nblk: int, kk: int, out: torch.Tensor | None) -> torch.Tensor:
+    B, _, H, _ = q.shape
+    if out is None:
+        return torch.empty((B, H, nblk, kk), dtype=torch.int32, device=q.device)
+    if out.shape != (B, H, nblk, kk) or out.dtype != torch.int32 or not out.is_contiguous():
+        raise ValueError("out must be a contiguous int32 [B, heads, nblk, k] tensor")
+    return out
 
 
 def route_k(nkv: int, sparsity: float) -> int:
@@ -172,13 +239,8 @@ def route(q: torch.Tensor, k: torch.Tensor, sparsity: float, block: int = BLOCK,
     kk = route_k(nblk, sparsity)
     if kk < 0:
         raise ValueError(f"sparsity {sparsity} outside [0, 1)")
-    ws_bytes = route_workspace_size(q, block)
-    if workspace is None:
-        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
-    if out is None:
-        out = torch.empty((B, H, nblk, kk), dtype=torch.int32, device=q.device)
-    elif out.shape != (B, H, nblk, kk) or out.dtype != torch.int32 or not out.is_contiguous():
-        raise ValueError("out must be a contiguous int32 [B, heads, nblk, k] tensor")
+    workspace = _workspace(q, workspace, block)
+    out = _route_out(q, nblk, kk, out)
     k_out = ctypes.c_int64(0)
     d = desc_of(q)
     _check("h3a_route", lib.h3a_route(_ptr(q), _ptr(k), ctypes.byref(d), float(sparsity), block, _ptr(out),
@@ -244,8 +306,9 @@ def attention_core(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, gamma_q: t
                    eps: float = 1e-6, workspace: torch.Tensor | None = None):
     """The whole per-layer core: prologue over Q/K, then dense attention
     (sparsity None) or router + block-sparse attention.  Returns (o, block_idx or None)."""
-    qn, kn = qk_norm_rope(q, k, gamma_q, gamma_k, grid, theta, eps)
-    blocks = None
-    if sparsity is not None:
-        blocks = route(qn, kn, sparsity, workspace=workspace)
+    if sparsity is None:
+        qn, kn = qk_norm_rope(q, k, gamma_q, gamma_k, grid, theta, eps)
+        return attention(qn, kn, v), None
+    qn, kn, ws = qk_norm_rope_pool(q, k, gamma_q, gamma_k, grid, theta, eps, workspace=workspace)
+    blocks = route_pooled(qn, sparsity, ws)
     return attention(qn, kn, v, blocks), blocks

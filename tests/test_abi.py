@@ -117,6 +117,41 @@ def test_route_validation():
 
 
 @NO_GPU
+def test_fused_prologue_and_pooled_route_validation():
+    lib = h3a.load()
+    d = _desc(N=8064)
+    grid = h3a.Grid(8, 24, 42)
+    ws = 2 * ((56 * 63 * 96 * 4 + 255) // 256 * 256)
+    kk = ctypes.c_int64()
+
+    def pro(q=GOOD, gq=GOOD, grid=grid, eps=1e-6, w=GOOD, wsb=ws, desc=None):
+        return lib.h3a_qk_norm_rope_pool(q, GOOD, ctypes.byref(desc or d), gq, GOOD, grid, 1e4, eps, GOOD, GOOD,
+                                         w, wsb, None)
+
+    assert pro(q=None) == 1
+    assert pro(q=MISALIGNED) == 1
+    assert pro(gq=None) == 1
+    assert pro(grid=h3a.Grid(8, 24, 41)) == 1          # T*H*W != N
+    assert pro(eps=-1.0) == 1
+    assert pro(desc=_desc(D=64)) == 2                   # head_dim != 96
+    assert pro(w=None) == 5
+    assert pro(wsb=ws - 1) == 5
+    assert pro(w=MISALIGNED) == 5
+
+    def rp(s=0.75, block=128, idx=GOOD, w=GOOD, wsb=ws, desc=None):
+        return lib.h3a_route_pooled(ctypes.byref(desc or d), s, block, idx, ctypes.byref(kk), w, wsb, None)
+
+    assert rp(s=1.0) == 1
+    assert rp(s=-0.1) == 1
+    assert rp(block=64) == 2
+    assert rp(idx=None) == 1
+    assert rp(idx=P(0x10002)) == 1
+    assert rp(w=None) == 5
+    assert rp(wsb=ws - 1) == 5
+    assert rp(desc=_desc(D=128)) == 2
+
+
+@NO_GPU
 def test_attention_validation():
     lib = h3a.load()
     d = _desc(N=8064)

@@ -73,3 +73,30 @@ def test_video5s_dense_and_sparse(orc):
 def test_video10s_sparse_and_dense(orc):
     w, d, ora_q, ora_k = _stage(orc, "video10s")
     _attention_checks(orc, w, d, ora_q, ora_k, 0.80, 2048)
+
+
+def test_video5s_fused_prologue_pool_route(orc):
+    """The fused prologue + pooling and the pooled router at 124,992 tokens, as
+    the bench runs them: bit-identical to the unfused calls (outputs and block
+    lists), the lists within the router rule of the oracle's, the outputs by the
+    prologue rule on sampled tokens."""
+    w = synth.WORKLOADS["video5s_sparse"]
+    d = synth.draw_workload("video5s_sparse")
+    g = w.grid
+    q, k = d["q"].cuda(), d["k"].cuda()
+    gq, gk = d["gamma_q"].cuda(), d["gamma_k"].cuda()
+    qo, ko, ws = h3a.qk_norm_rope_pool(q, k, gq, gk, g)
+    idx = h3a.route_pooled(qo, 0.75, ws)
+    qu, ku = h3a.qk_norm_rope(q, k, gq, gk, g)
+    idx_u = h3a.route(qu, ku, 0.75)
+    torch.cuda.synchronize()
+    assert torch.equal(qo.view(torch.int16), qu.view(torch.int16))
+    assert torch.equal(ko.view(torch.int16), ku.view(torch.int16))
+    assert torch.equal(idx, idx_u)
+    del qu, ku, idx_u, q, k
+    tok = synth.sample_rows(1, 1, w.N, 2048, seed=7).numpy()
+    for x, gam, out in ((d["q"], d["gamma_q"], qo), (d["k"], d["gamma_k"], ko)):
+        want = orc.round_bf16(orc.qk_norm_rope_tokens(x, gam.numpy(), g, tok))
+        check_prologue(bits(out[0, torch.as_tensor(tok).cuda()]), want, "video5s fused prologue")
+    ora_idx, ora_sc = orc.route(bits(qo), bits(ko), 0.75)
+    check_router(idx.cpu().numpy(), ora_idx, ora_sc, "video5s pooled router")
