@@ -196,7 +196,10 @@ def run_gpu(args, rank, world, local):
     dev = torch.device("cuda", local)
     q, k, v = (d[n].to(dev) for n in "qkv")
     gq, gk = d["gamma_q"].to(dev), d["gamma_k"].to(dev)
-    qn, kn = torch.empty_like(q), torch.empty_like(k)
+    # the 3D RoPE prologue is defined for 96 channels; a 128-wide workload runs
+    # the router (with its own pooling) and attention on the inputs directly
+    wide = w.head_dim != 96
+    qn, kn = (q, k) if wide else (torch.empty_like(q), torch.empty_like(k))
     o_dense, o_sparse = torch.empty_like(q), torch.empty_like(q)
     nblk = (N + 127) // 128
     kk = h3a.route_k(nblk, SPARSITY)
@@ -209,10 +212,14 @@ def run_gpu(args, rank, world, local):
     def step(ev=None):
         if ev is not None:
             ev[0].record(stream)
-        h3a.qk_norm_rope_pool(q, k, gq, gk, grid, workspace=ws, out=(qn, kn))
+        if not wide:
+            h3a.qk_norm_rope_pool(q, k, gq, gk, grid, workspace=ws, out=(qn, kn))
         if ev is not None:
             ev[1].record(stream)
-        h3a.route_pooled(qn, SPARSITY, ws, out=blocks)
+        if wide:
+            h3a.route(qn, kn, SPARSITY, workspace=ws, out=blocks)
+        else:
+            h3a.route_pooled(qn, SPARSITY, ws, out=blocks)
         if ev is not None:
             ev[2].record(stream)
         h3a.attention(qn, kn, v, blocks, out=o_sparse)
@@ -227,8 +234,8 @@ def run_gpu(args, rank, world, local):
     torch.cuda.synchronize()
     if h3a.last_device_error() != 0:
         raise RuntimeError("device-side timeout during warm-up")
-    flops_dense = attention_flops(N, heads, B)
-    flops_sparse = attention_flops(N, heads, B, blocks=blocks.cpu().numpy())
+    flops_dense = attention_flops(N, heads, B, d=w.head_dim)
+    flops_sparse = attention_flops(N, heads, B, d=w.head_dim, blocks=blocks.cpu().numpy())
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
     barrier(world)
@@ -249,7 +256,7 @@ def run_gpu(args, rank, world, local):
     # for comparison, outside the timed region: the separate prologue and the
     # router with its own pooling pass
     sep = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(5)]
-    for i in range(6):
+    for i in range(0 if wide else 6):
         e = sep[i - 1] if i > 0 else None
         if e is not None:
             e[0].record(stream)
@@ -260,8 +267,12 @@ def run_gpu(args, rank, world, local):
         if e is not None:
             e[2].record(stream)
     torch.cuda.synchronize()
-    kern_ms["prologue"] = allreduce_max(float(np.mean([e[0].elapsed_time(e[1]) for e in sep])), world)
-    kern_ms["router"] = allreduce_max(float(np.mean([e[1].elapsed_time(e[2]) for e in sep])), world)
+    if wide:
+        kern_ms["prologue"] = kern_ms["prologue_pool"] = 0.0
+        kern_ms["router"] = kern_ms["router_scores"]
+    else:
+        kern_ms["prologue"] = allreduce_max(float(np.mean([e[0].elapsed_time(e[1]) for e in sep])), world)
+        kern_ms["router"] = allreduce_max(float(np.mean([e[1].elapsed_time(e[2]) for e in sep])), world)
 
     # end to end through the public API with host buffers
     e2e = None
@@ -301,9 +312,11 @@ def run_gpu(args, rank, world, local):
     pk, pk_src = peaks()
     dense_tflops = flops_dense / (kern_ms["attention_dense"] * 1e-3) / 1e12
     sparse_tflops = flops_sparse / (kern_ms["attention_sparse"] * 1e-3) / 1e12
-    pro_gbs = prologue_bytes(N, heads, B) / (kern_ms["prologue"] * 1e-3) / 1e9
-    router_gbs = router_bytes(N, heads, B) / (kern_ms["router"] * 1e-3) / 1e9
-    fused_gbs = (prologue_bytes(N, heads, B) + pooled_bytes(N, heads, B)) / (kern_ms["prologue_pool"] * 1e-3) / 1e9
+    D = w.head_dim
+    router_gbs = router_bytes(N, heads, B, D) / (kern_ms["router"] * 1e-3) / 1e9
+    if not wide:
+        pro_gbs = prologue_bytes(N, heads, B) / (kern_ms["prologue"] * 1e-3) / 1e9
+        fused_gbs = (prologue_bytes(N, heads, B) + pooled_bytes(N, heads, B)) / (kern_ms["prologue_pool"] * 1e-3) / 1e9
     # the sparse path's routing cost: scores + top-k, plus what pooling adds to the prologue
     route_cost = kern_ms["router_scores"] + max(0.0, kern_ms["prologue_pool"] - kern_ms["prologue"])
     traffic = load_traffic()
@@ -322,12 +335,14 @@ def run_gpu(args, rank, world, local):
         "dtype": "bf16",
         "data": "synthetic",
         "config": {
-            "workload": f"{w.name}: B={B}, {heads} heads x 96, grid {grid[0]}x{grid[1]}x{grid[2]} = {N:,} tokens "
-                        f"per GPU; prologue with block pooling + router scores/top-k (sparsity {SPARSITY}, "
-                        f"k={kk}/{nblk}) + sparse + dense attention",
-            "tokens": N, "heads": heads, "head_dim": 96, "batch_per_gpu": B, "sparsity": SPARSITY,
+            "workload": f"{w.name}: B={B}, {heads} heads x {D}, grid {grid[0]}x{grid[1]}x{grid[2]} = {N:,} tokens "
+                        f"per GPU; " + (f"router with its own pooling (sparsity {SPARSITY}, k={kk}/{nblk}) + sparse + "
+                                        "dense attention (no prologue: its 3D RoPE is defined for 96 channels)" if wide
+                                        else f"prologue with block pooling + router scores/top-k (sparsity {SPARSITY}, "
+                                        f"k={kk}/{nblk}) + sparse + dense attention"),
+            "tokens": N, "heads": heads, "head_dim": D, "batch_per_gpu": B, "sparsity": SPARSITY,
             "parallelism": f"dp{world} (independent clips per GPU)",
-            "l2": f"inputs larger than L2 (Q, K, V {B * N * heads * 96 * 2 / 1e9:.2f} GB each); no explicit flush",
+            "l2": f"inputs larger than L2 (Q, K, V {B * N * heads * D * 2 / 1e9:.2f} GB each); no explicit flush",
         },
         "roofline": {
             "kernel": "attention_kernel (dense)",
@@ -339,10 +354,12 @@ def run_gpu(args, rank, world, local):
             "peak_source": f"{pk_src} bf16 sustained (kernel timed inside a long step)",
             "frac_of_burst": round(dense_tflops / pk["bf16_tflops"], 4),
             "frac_of_spec_2250": round(dense_tflops / 2250.0, 4),
-            "traffic": traffic.get("attention_dense", {}).get("bytes_per_launch"),
+            "traffic": None if wide else traffic.get("attention_dense", {}).get("bytes_per_launch"),
             "algorithmic_flops_per_launch": flops_dense,
         },
-        "kernels": {
+        "kernels": ({
+            "router": {"ms": round(kern_ms["router"], 4), "pool_read_GB/s": round(router_gbs, 1)},
+        } if wide else {
             "prologue_pool": {"ms": round(kern_ms["prologue_pool"], 4), "GB/s": round(fused_gbs, 1),
                               "frac_hbm": round(fused_gbs / pk["hbm_gbs"], 4),
                               "frac_8TBs": round(fused_gbs / 8000.0, 4),
@@ -354,6 +371,7 @@ def run_gpu(args, rank, world, local):
                                                "traffic": traffic.get("prologue", {}).get("bytes_per_launch")},
             "separate_router_untimed_step": {"ms": round(kern_ms["router"], 4),
                                              "pool_read_GB/s": round(router_gbs, 1)},
+        }) | {
             "attention_sparse": {"ms": round(kern_ms["attention_sparse"], 3), "TFLOP/s": round(sparse_tflops, 2),
                                  "effective_dense_equiv_TFLOP/s":
                                      round(flops_dense / (kern_ms["attention_sparse"] * 1e-3) / 1e12, 2),
@@ -377,8 +395,11 @@ def _oracle_inputs(d, w, sparsity):
     import oracle
 
     oracle.build()
-    qb = oracle.qk_norm_rope_bf16(d["q"], d["gamma_q"].numpy(), w.grid)
-    kb = oracle.qk_norm_rope_bf16(d["k"], d["gamma_k"].numpy(), w.grid)
+    if w.head_dim != 96:  # no prologue at this width: attention sees the inputs as drawn
+        qb, kb = d["q"], d["k"]
+    else:
+        qb = oracle.qk_norm_rope_bf16(d["q"], d["gamma_q"].numpy(), w.grid)
+        kb = oracle.qk_norm_rope_bf16(d["k"], d["gamma_k"].numpy(), w.grid)
     idx, _ = oracle.route(qb, kb, sparsity)
     return qb, kb, idx
 
@@ -397,7 +418,7 @@ def _oracle_sample(d, w, qb, kb, idx, rows):
     lens[-1] = N - (nblk - 1) * 128
     bh, n = rows // N, rows % N
     sparse_keys = lens[idx.reshape(-1, nblk, idx.shape[-1])[bh, n // 128]].sum(axis=-1).sum()
-    flops = 4.0 * 96 * (len(rows) * N + sparse_keys)
+    flops = 4.0 * w.head_dim * (len(rows) * N + sparse_keys)
     return dt, flops
 
 

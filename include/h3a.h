@@ -10,7 +10,10 @@
  *   - Tensors are bf16 (raw 16-bit words), laid out [B, N, heads, head_dim]
  *     with head_dim contiguous and element strides given by h3a_qkv_desc.
  *     Token n of the (T, H, W) grid is n = (t*H + h)*W + w.
- *   - head_dim must be 96 (hidden 5376 / 56 heads), block must be 128.
+ *   - head_dim must be 96 (hidden 5376 / 56 heads); the router and attention
+ *     also take 128 (SubBlock's stated head size; the same hidden width as
+ *     42 heads), the prologue does not (its 3D RoPE layout is defined for 96
+ *     channels).  block must be 128.
  *   - All pointers are DEVICE pointers owned by the caller, 16-byte aligned;
  *     strides are multiples of 8 elements (16 bytes).  The library never
  *     allocates or frees device memory; the router's scratch is a caller
@@ -38,7 +41,7 @@ typedef struct CUstream_st* h3a_stream_t; /* a cudaStream_t; NULL = legacy defau
 typedef enum {
     H3A_OK = 0,
     H3A_ERR_INVALID_ARG = 1, /* null/misaligned pointer, inconsistent sizes, bad sparsity */
-    H3A_ERR_UNSUPPORTED = 2, /* head_dim != 96, block != 128, sizes beyond the int32 index range */
+    H3A_ERR_UNSUPPORTED = 2, /* head_dim not supported by the call, block != 128, sizes beyond int32 range */
     H3A_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed (see h3a_last_cuda_error_string) */
     H3A_ERR_TIMEOUT = 4,     /* a bounded device-side wait expired; results are undefined */
     H3A_ERR_WORKSPACE = 5    /* router workspace null or too small */
@@ -82,9 +85,9 @@ h3a_status h3a_qk_norm_rope(const void* q, const void* k, const h3a_qkv_desc* d,
  * Returns -1 if sparsity is outside [0, 1) or nkv < 1. */
 int64_t h3a_route_k(int64_t nkv, double sparsity);
 
-/* Bytes of device workspace h3a_route needs: two fp32 [B, heads, nblk, 96]
- * pooled tensors, nblk = ceil(N / block).  Returns INVALID_ARG/UNSUPPORTED
- * for bad descriptors. */
+/* Bytes of device workspace h3a_route needs: two fp32 [B, heads, nblk,
+ * head_dim] pooled tensors, nblk = ceil(N / block), head_dim 96 or 128.
+ * Returns INVALID_ARG/UNSUPPORTED for bad descriptors. */
 h3a_status h3a_route_workspace_size(const h3a_qkv_desc* d, int32_t block, size_t* bytes);
 
 /* Blockwise KV-block router.
@@ -93,15 +96,15 @@ h3a_status h3a_route_workspace_size(const h3a_qkv_desc* d, int32_t block, size_t
  * sparse router prunes the KV blocks, sparsity 0.75 or 0.80); pooling,
  * scoring and selection as fixed by the problem statement:
  *   qbar_i, kbar_j = fp32 means of the 128-token blocks (the tail block over
- *   its real length), score S_ij = (qbar_i . kbar_j) / sqrt(96) in fp32,
+ *   its real length), score S_ij = (qbar_i . kbar_j) / sqrt(head_dim) in fp32,
  *   per (b, h, i) keep the k highest scores, ties to the lower j.
  * q, k       : prologue outputs (device, bf16, layout d).
  * block_idx  : device int32 [B, heads, nblk, k], each row ascending.
  * k_out      : host; receives k (may be NULL).
  * workspace  : device, at least h3a_route_workspace_size bytes, 16-B aligned.
  * Errors: INVALID_ARG for null pointers or sparsity outside [0, 1);
- * UNSUPPORTED for block != 128 or head_dim != 96; WORKSPACE if the
- * workspace is null or ws_bytes is too small. */
+ * UNSUPPORTED for block != 128 or head_dim other than 96 / 128; WORKSPACE if
+ * the workspace is null or ws_bytes is too small. */
 h3a_status h3a_route(const void* q, const void* k, const h3a_qkv_desc* d, double sparsity,
                      int32_t block, int32_t* block_idx, int64_t* k_out, void* workspace,
                      size_t ws_bytes, h3a_stream_t stream);
@@ -131,7 +134,8 @@ h3a_status h3a_qk_norm_rope_pool(const void* q, const void* k, const h3a_qkv_des
  * h3a_qk_norm_rope_pool left in the workspace (same source and rule as
  * h3a_route).  d describes the Q/K tensors that were pooled; block_idx,
  * k_out and the result are those of h3a_route on the prologue's outputs.
- * The workspace is only read.  Errors: as h3a_route. */
+ * The workspace is only read.  Errors: as h3a_route, and UNSUPPORTED for a
+ * head_dim other than 96 (the prologue's only width). */
 h3a_status h3a_route_pooled(const h3a_qkv_desc* d, double sparsity, int32_t block,
                             int32_t* block_idx, int64_t* k_out, const void* workspace,
                             size_t ws_bytes, h3a_stream_t stream);
@@ -175,8 +179,8 @@ h3a_status h3a_route_noalloc(const void* q, const void* k, const h3a_qkv_desc* d
  * Tensor-core path: TMA tiles, tcgen05.mma with TMEM accumulators, fp32
  * online softmax, one rounding of O to bf16.
  * Errors: INVALID_ARG for null/misaligned pointers or k_blocks outside
- * [1, nblk] in sparse mode; UNSUPPORTED for head_dim != 96, block != 128, or
- * N >= 2^31. */
+ * [1, nblk] in sparse mode; UNSUPPORTED for head_dim other than 96 / 128,
+ * block != 128, or N >= 2^31. */
 h3a_status h3a_attention(const void* q, const void* k, const void* v, const h3a_qkv_desc* d,
                          const int32_t* block_idx, int32_t k_blocks, int32_t block, float scale,
                          void* o, h3a_stream_t stream);

@@ -30,7 +30,9 @@
 //               TMEM, V as an MN-major operand).  Order per step j:
 //               PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1), so each softmax group
 //               waits only on its own tile's chain.
-// TMEM columns: S_0 [0,128), S_1 [128,256), O_0 [256,352), O_1 [352,448).
+// TMEM columns: S_0 [0,128), S_1 [128,256), O_0 [256,352), O_1 [352,448) at
+// head_dim 96; the same kernel is instantiated for head_dim 128 (O_0
+// [256,384), O_1 [384,512), four 32-channel chunks per tile, 2-stage rings).
 // Every mbarrier wait is bounded (timeout + CTA abort flag); a timeout sets the
 // device status word instead of hanging or trapping.
 #include <cuda_bf16.h>
@@ -44,16 +46,31 @@ namespace {
 constexpr int kSoftmaxWarps = 16;                  // 4 warpgroups: (tile, column half)
 constexpr int kProducerWarp = 16, kMmaWarp = 17;
 constexpr int kThreads = 32 * (kSoftmaxWarps + 2);  // 576
-constexpr int kStages = 3;
 constexpr int kChunkBytes = 128 * 64;        // 128 rows x 32 bf16, 64-byte swizzle
-constexpr int kTileBytes = 3 * kChunkBytes;  // 128 x 96 bf16
 constexpr uint32_t kTmemCols = 512;
-// TMEM column of S_t / O_t
+// TMEM column of S_t
 __host__ __device__ constexpr uint32_t col_s(int t) { return t ? 128u : 0u; }
-__host__ __device__ constexpr uint32_t col_o(int t) { return t ? 352u : 256u; }
 constexpr uint32_t kSwizzle64 = 4;
 
+// Geometry per head dimension D (96, or 128 -- SubBlock's stated head size):
+// a 128-row tile is D/32 swizzled 32-channel chunks; O_t takes D TMEM columns
+// (O_0 [256, 256+D), O_1 [256+D, 256+2D)); at D = 128 the K and V rings keep
+// two stages each so that Q tiles and rings fit in 227 KB of shared memory.
+template <int D>
+struct Geo {
+    static_assert(D == 96 || D == 128, "head_dim 96 or 128");
+    static constexpr int kChunks = D / 32;
+    static constexpr int kTileBytes = kChunks * kChunkBytes;
+    static constexpr int kStages = D == 96 ? 3 : 2;
+    static constexpr int kKSteps = D / 16;  // QK^T k-steps of 16
+    static constexpr int kHalf = D / 2;     // O columns per softmax half
+    __host__ __device__ static constexpr uint32_t col_o(int t) { return 256u + (t ? D : 0); }
+};
+
+template <int D>
 struct AttnSmem {
+    static constexpr int kStages = Geo<D>::kStages;
+    static constexpr int kTileBytes = Geo<D>::kTileBytes;
     uint8_t q[2][kTileBytes];
     uint8_t k[kStages][kTileBytes];
     uint8_t v[kStages][kTileBytes];
@@ -71,7 +88,16 @@ struct AttnSmem {
     int never;  // stays 0: abort flag for waits that must ignore an abort
 };
 
-constexpr size_t kSmemBytes = sizeof(AttnSmem) + 1024;  // + alignment slack
+// tcgen05.ld / st of 16 or 32 columns, chosen by the register array's size.
+__device__ __forceinline__ void tmem_ld_n(uint32_t a, uint32_t (&r)[16]) { tmem_ld_x16(a, r); }
+__device__ __forceinline__ void tmem_ld_n(uint32_t a, uint32_t (&r)[32]) { tmem_ld_x32(a, r); }
+__device__ __forceinline__ void tmem_wait_ld_n(uint32_t (&r)[16]) { tmem_wait_ld_x16(r); }
+__device__ __forceinline__ void tmem_wait_ld_n(uint32_t (&r)[32]) { tmem_wait_ld_x32(r); }
+__device__ __forceinline__ void tmem_st_n(uint32_t a, const uint32_t (&r)[16]) { tmem_st_x16(a, r); }
+__device__ __forceinline__ void tmem_st_n(uint32_t a, const uint32_t (&r)[32]) { tmem_st_x32(a, r); }
+
+template <int D>
+constexpr size_t smem_bytes() { return sizeof(AttnSmem<D>) + 1024; }  // + alignment slack
 
 struct AttnArgs {
     __nv_bfloat16* o;
@@ -95,7 +121,7 @@ __device__ __forceinline__ void raise_timeout(const AttnArgs& a, volatile int* a
 // per tcgen05.mma -- computing descriptors per MMA made the issue thread,
 // not the tensor core, the bottleneck.
 //
-// K-major 128 x 96 tile (three swizzled 32-column chunks of 64-byte rows):
+// K-major 128 x D tile (D/32 swizzled 32-column chunks of 64-byte rows):
 // k-step s covers columns [16s, 16s + 16).
 __device__ __forceinline__ uint64_t kmajor_base(const uint8_t* tile) {
     return smem_desc(smem_u32(tile), 16, 512, kSwizzle64);
@@ -104,14 +130,15 @@ __host__ __device__ constexpr uint32_t kmajor_step(int s) {
     return static_cast<uint32_t>(((s >> 1) * kChunkBytes + (s & 1) * 32) >> 4);
 }
 
-// The same [128 kv rows x 96] tile read as an MN-major operand (N = 96 along
+// The same [128 kv rows x D] tile read as an MN-major operand (N = D along
 // the contiguous dimension, K = kv rows): k-step s covers rows [16s, 16s + 16).
 __device__ __forceinline__ uint64_t mnmajor_base(const uint8_t* tile) {
     return smem_desc(smem_u32(tile), kChunkBytes, 512, kSwizzle64);
 }
 __host__ __device__ constexpr uint32_t mnmajor_step(int s) { return static_cast<uint32_t>((s * 16 * 64) >> 4); }
 
-constexpr uint32_t kStageStep = kTileBytes >> 4;  // descriptor distance between ring stages
+template <int D>
+constexpr uint32_t stage_step() { return Geo<D>::kTileBytes >> 4; }  // descriptor distance between ring stages
 
 struct KvPlan {
     int kv0, kv1;
@@ -126,7 +153,8 @@ __device__ __forceinline__ KvPlan kv_plan(const int32_t* l0, const int32_t* l1, 
     return p;
 }
 
-__device__ void producer(AttnSmem& sm, const AttnArgs& a, const CUtensorMap* tq, const CUtensorMap* tk,
+template <int D>
+__device__ void producer(AttnSmem<D>& sm, const AttnArgs& a, const CUtensorMap* tq, const CUtensorMap* tk,
                          const CUtensorMap* tv, int b, int h, int qb0, bool has1, const int32_t* l0,
                          const int32_t* l1, volatile int* abort_flag) {
     prefetch_tensor_map(tq);
@@ -134,8 +162,8 @@ __device__ void producer(AttnSmem& sm, const AttnArgs& a, const CUtensorMap* tq,
     prefetch_tensor_map(tv);
     const int ntiles = has1 ? 2 : 1;
     for (int t = 0; t < ntiles; ++t) {
-        mbar_arrive_expect_tx(&sm.q_full[t], kTileBytes);
-        for (int c = 0; c < 3; ++c)
+        mbar_arrive_expect_tx(&sm.q_full[t], Geo<D>::kTileBytes);
+        for (int c = 0; c < Geo<D>::kChunks; ++c)
             tma_load_4d(sm.q[t] + c * kChunkBytes, tq, &sm.q_full[t], 32 * c, h, (qb0 + t) * 128, b);
     }
     uint32_t ks = 0, kph = 0, vs = 0, vph = 0;
@@ -151,12 +179,12 @@ __device__ void producer(AttnSmem& sm, const AttnArgs& a, const CUtensorMap* tq,
                 break;
             }
             const int kv = u ? p.kv1 : p.kv0;
-            mbar_arrive_expect_tx(&sm.k_full[ks], kTileBytes);
-            for (int c = 0; c < 3; ++c)
+            mbar_arrive_expect_tx(&sm.k_full[ks], Geo<D>::kTileBytes);
+            for (int c = 0; c < Geo<D>::kChunks; ++c)
                 tma_load_4d(sm.k[ks] + c * kChunkBytes, tk, &sm.k_full[ks], 32 * c, h, kv * 128, b);
             k_issued |= 1u << ks;
             k_par = (k_par & ~(1u << ks)) | (kph << ks);
-            if (++ks == kStages) {
+            if (++ks == Geo<D>::kStages) {
                 ks = 0;
                 kph ^= 1u;
             }
@@ -167,12 +195,12 @@ __device__ void producer(AttnSmem& sm, const AttnArgs& a, const CUtensorMap* tq,
                 break;
             }
             const int kv = u ? p.kv1 : p.kv0;
-            mbar_arrive_expect_tx(&sm.v_full[vs], kTileBytes);
-            for (int c = 0; c < 3; ++c)
+            mbar_arrive_expect_tx(&sm.v_full[vs], Geo<D>::kTileBytes);
+            for (int c = 0; c < Geo<D>::kChunks; ++c)
                 tma_load_4d(sm.v[vs] + c * kChunkBytes, tv, &sm.v_full[vs], 32 * c, h, kv * 128, b);
             v_issued |= 1u << vs;
             v_par = (v_par & ~(1u << vs)) | (vph << vs);
-            if (++vs == kStages) {
+            if (++vs == Geo<D>::kStages) {
                 vs = 0;
                 vph ^= 1u;
             }
@@ -182,7 +210,7 @@ __device__ void producer(AttnSmem& sm, const AttnArgs& a, const CUtensorMap* tq,
     // Drain: every load issued must have landed before the CTA may exit.
     volatile int* never = &sm.never;
     for (int t = 0; t < ntiles; ++t) mbar_wait(&sm.q_full[t], 0u, never, a.timeout_ns);
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < Geo<D>::kStages; ++s) {
         if ((k_issued >> s) & 1u) mbar_wait(&sm.k_full[s], (k_par >> s) & 1u, never, a.timeout_ns);
         if ((v_issued >> s) & 1u) mbar_wait(&sm.v_full[s], (v_par >> s) & 1u, never, a.timeout_ns);
     }
@@ -194,13 +222,14 @@ struct MmaState {
     uint64_t dq[2], dk, dv;  // base descriptors: Q tiles, K stage 0, V stage 0
 };
 
-__device__ __forceinline__ bool issue_qk(AttnSmem& sm, const AttnArgs& a, MmaState& st, uint32_t tmem, int t,
+template <int D>
+__device__ __forceinline__ bool issue_qk(AttnSmem<D>& sm, const AttnArgs& a, MmaState& st, uint32_t tmem, int t,
                                          const KvPlan& p, volatile int* abort_flag) {
     uint32_t stage;
     if (t == 0 || !p.shared) {
         if (!mbar_wait(&sm.k_full[st.ks], st.kph, abort_flag, a.timeout_ns)) return false;
         stage = st.ks;
-        if (++st.ks == kStages) {
+        if (++st.ks == Geo<D>::kStages) {
             st.ks = 0;
             st.kph ^= 1u;
         }
@@ -211,22 +240,23 @@ __device__ __forceinline__ bool issue_qk(AttnSmem& sm, const AttnArgs& a, MmaSta
     tc_fence_after_sync();
     constexpr uint32_t idesc = idesc_bf16_f32(128, 128, 0, 0);
     const uint64_t dq = st.dq[t];
-    const uint64_t dk = st.dk + stage * kStageStep;
+    const uint64_t dk = st.dk + stage * stage_step<D>();
     const uint32_t d = tmem + col_s(t);
 #pragma unroll
-    for (int s = 0; s < 6; ++s) mma_ss(d, dq + kmajor_step(s), dk + kmajor_step(s), idesc, s > 0 ? 1u : 0u);
+    for (int s = 0; s < Geo<D>::kKSteps; ++s) mma_ss(d, dq + kmajor_step(s), dk + kmajor_step(s), idesc, s > 0 ? 1u : 0u);
     tc_commit(&sm.s_full[t]);
     if (t == 1 || !p.shared) tc_commit(&sm.k_empty[stage]);
     return true;
 }
 
-__device__ __forceinline__ bool issue_pv(AttnSmem& sm, const AttnArgs& a, MmaState& st, uint32_t tmem, int t,
+template <int D>
+__device__ __forceinline__ bool issue_pv(AttnSmem<D>& sm, const AttnArgs& a, MmaState& st, uint32_t tmem, int t,
                                          const KvPlan& p, bool first, volatile int* abort_flag) {
     uint32_t stage;
     if (t == 0 || !p.shared) {
         if (!mbar_wait(&sm.v_full[st.vs], st.vph, abort_flag, a.timeout_ns)) return false;
         stage = st.vs;
-        if (++st.vs == kStages) {
+        if (++st.vs == Geo<D>::kStages) {
             st.vs = 0;
             st.vph ^= 1u;
         }
@@ -235,9 +265,9 @@ __device__ __forceinline__ bool issue_pv(AttnSmem& sm, const AttnArgs& a, MmaSta
     }
     if (t == 0) st.v_stage_t0 = stage;
     tc_fence_after_sync();
-    constexpr uint32_t idesc = idesc_bf16_f32(128, 96, 0, 1);
-    const uint64_t dv = st.dv + stage * kStageStep;
-    const uint32_t d = tmem + col_o(t), pa = tmem + col_s(t);
+    constexpr uint32_t idesc = idesc_bf16_f32(128, D, 0, 1);
+    const uint64_t dv = st.dv + stage * stage_step<D>();
+    const uint32_t d = tmem + Geo<D>::col_o(t), pa = tmem + col_s(t);
     // keys 0..63: P at S columns [0, 32); keys 64..127: P at S columns [64, 96)
     mma_ts(d, pa, dv, idesc, first ? 0u : 1u);
 #pragma unroll
@@ -246,7 +276,8 @@ __device__ __forceinline__ bool issue_pv(AttnSmem& sm, const AttnArgs& a, MmaSta
     return true;
 }
 
-__device__ void mma_issuer(AttnSmem& sm, const AttnArgs& a, uint32_t tmem, bool has1, const int32_t* l0,
+template <int D>
+__device__ void mma_issuer(AttnSmem<D>& sm, const AttnArgs& a, uint32_t tmem, bool has1, const int32_t* l0,
                            const int32_t* l1, volatile int* abort_flag) {
     const int ntiles = has1 ? 2 : 1;
     MmaState st;
@@ -260,7 +291,7 @@ __device__ void mma_issuer(AttnSmem& sm, const AttnArgs& a, uint32_t tmem, bool 
     KvPlan p = kv_plan(l0, l1, has1, 0);
     KvPlan pn = a.n_iter > 1 ? kv_plan(l0, l1, has1, 1) : p;
     if (ok)
-        for (int t = 0; t < ntiles && ok; ++t) ok = issue_qk(sm, a, st, tmem, t, p, abort_flag);
+        for (int t = 0; t < ntiles && ok; ++t) ok = issue_qk<D>(sm, a, st, tmem, t, p, abort_flag);
     for (int j = 0; j < a.n_iter && ok; ++j) {
         const bool more = j + 1 < a.n_iter;
         const KvPlan pnn = (j + 2 < a.n_iter) ? kv_plan(l0, l1, has1, j + 2) : pn;
@@ -270,12 +301,12 @@ __device__ void mma_issuer(AttnSmem& sm, const AttnArgs& a, uint32_t tmem, bool 
                 break;
             }
             tc_fence_after_sync();
-            if (!issue_pv(sm, a, st, tmem, t, p, j == 0, abort_flag)) {
+            if (!issue_pv<D>(sm, a, st, tmem, t, p, j == 0, abort_flag)) {
                 ok = false;
                 break;
             }
             if (more) {
-                if (!issue_qk(sm, a, st, tmem, t, pn, abort_flag)) ok = false;
+                if (!issue_qk<D>(sm, a, st, tmem, t, pn, abort_flag)) ok = false;
             } else {
                 tc_commit(&sm.o_done[t]);
             }
@@ -319,14 +350,16 @@ __device__ __forceinline__ float exp_store_half(const uint32_t (&s)[2][32], floa
 // block: thread r owns row r (TMEM lane r) of that half.  The two halves of a
 // row run in two warpgroups and agree on the row's reference max through
 // shared memory and a bounded mbarrier wait per block.
-__device__ void softmax_group(AttnSmem& sm, const AttnArgs& a, uint32_t tmem, int t, int hf, int b, int h, int qb,
+template <int D>
+__device__ void softmax_group(AttnSmem<D>& sm, const AttnArgs& a, uint32_t tmem, int t, int hf, int b, int h, int qb,
                               const int32_t* list, volatile int* abort_flag) {
     const int lane = threadIdx.x & 31;
     const int quarter = (threadIdx.x >> 5) & 3;  // TMEM lanes [32*quarter, 32*quarter + 32)
     const int row = quarter * 32 + lane;
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t tS = tmem + lane_addr + col_s(t) + 64u * hf;
-    const uint32_t tO = tmem + lane_addr + col_o(t) + 48u * hf;
+    const uint32_t tO = tmem + lane_addr + Geo<D>::col_o(t) + static_cast<uint32_t>(Geo<D>::kHalf) * hf;
+    constexpr int kRest = Geo<D>::kHalf - 32;  // O columns of the half beyond the first 32 (16 or 32)
     const float c = a.scale_log2;
     float m_used = -INFINITY;  // row reference max of scaled logits (log2 units)
     float l = 0.f;             // this half's running sum of P
@@ -397,17 +430,17 @@ __device__ void softmax_group(AttnSmem& sm, const AttnArgs& a, uint32_t tmem, in
                     m_used = mx;
                 }
                 l = l * alpha + exp_store_half(s, c, m_used, tS, nullptr);
-                uint32_t o[32], o2[16];
+                uint32_t o[32], o2[kRest];
                 tmem_ld_x32(tO, o);
-                tmem_ld_x16(tO + 32, o2);
+                tmem_ld_n(tO + 32, o2);
                 tmem_wait_ld_x32(o);
-                tmem_wait_ld_x16(o2);
+                tmem_wait_ld_n(o2);
 #pragma unroll
                 for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
 #pragma unroll
-                for (int i = 0; i < 16; ++i) o2[i] = __float_as_uint(__uint_as_float(o2[i]) * alpha);
+                for (int i = 0; i < kRest; ++i) o2[i] = __float_as_uint(__uint_as_float(o2[i]) * alpha);
                 tmem_st_x32(tO, o);
-                tmem_st_x16(tO + 32, o2);
+                tmem_st_n(tO + 32, o2);
             } else {
                 l += ps;
             }
@@ -435,33 +468,35 @@ __device__ void softmax_group(AttnSmem& sm, const AttnArgs& a, uint32_t tmem, in
     tc_fence_after_sync();
     const float inv_l = 1.0f / (l + sm.lsum[t][hf ^ 1][row]);
     const int n = qb * 128 + row;
-    uint32_t o[32], o2[16];
+    uint32_t o[32], o2[kRest];
     tmem_ld_x32(tO, o);
-    tmem_ld_x16(tO + 32, o2);
+    tmem_ld_n(tO + 32, o2);
     tmem_wait_ld_x32(o);
-    tmem_wait_ld_x16(o2);
+    tmem_wait_ld_n(o2);
     if (n < a.N) {
         __nv_bfloat16* dst = a.o + static_cast<int64_t>(b) * a.sb + static_cast<int64_t>(n) * a.sn +
-                             static_cast<int64_t>(h) * a.sh + 48 * hf;
-        uint32_t w[24];
+                             static_cast<int64_t>(h) * a.sh + Geo<D>::kHalf * hf;
+        uint32_t w[Geo<D>::kHalf / 2];
 #pragma unroll
         for (int i = 0; i < 16; ++i)
             w[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
+        for (int i = 0; i < kRest / 2; ++i)
             w[16 + i] = pack_bf16x2(__uint_as_float(o2[2 * i]) * inv_l, __uint_as_float(o2[2 * i + 1]) * inv_l);
         uint4* d4 = reinterpret_cast<uint4*>(dst);
 #pragma unroll
-        for (int i = 0; i < 6; ++i) d4[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+        for (int i = 0; i < Geo<D>::kHalf / 8; ++i)
+            d4[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
     }
 }
 
+template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     attention_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                      const __grid_constant__ CUtensorMap tv, const AttnArgs a) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t base = smem_u32(smem_raw);
-    AttnSmem& sm = *reinterpret_cast<AttnSmem*>(smem_raw + (((base + 1023u) & ~1023u) - base));
+    AttnSmem<D>& sm = *reinterpret_cast<AttnSmem<D>*>(smem_raw + (((base + 1023u) & ~1023u) - base));
 
     const int warp = threadIdx.x >> 5;
     const int pair = blockIdx.x % a.npairs;
@@ -482,7 +517,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&sm.lbar[t], 8);
             mbar_init(&sm.o_done[t], 1);
         }
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < Geo<D>::kStages; ++s) {
             mbar_init(&sm.k_full[s], 1);
             mbar_init(&sm.k_empty[s], 1);
             mbar_init(&sm.v_full[s], 1);
@@ -504,13 +539,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     volatile int* abort_flag = &sm.abort_flag;
 
     if (warp == kProducerWarp) {
-        if ((threadIdx.x & 31) == 0) producer(sm, a, &tq, &tk, &tv, b, h, qb0, has1, l0, l1, abort_flag);
+        if ((threadIdx.x & 31) == 0) producer<D>(sm, a, &tq, &tk, &tv, b, h, qb0, has1, l0, l1, abort_flag);
     } else if (warp == kMmaWarp) {
-        if ((threadIdx.x & 31) == 0) mma_issuer(sm, a, tmem, has1, l0, l1, abort_flag);
+        if ((threadIdx.x & 31) == 0) mma_issuer<D>(sm, a, tmem, has1, l0, l1, abort_flag);
     } else {
         const int wg = warp >> 2;  // softmax warpgroup: tile wg / 2, column half wg % 2
         const int t = wg >> 1, hf = wg & 1;
-        if (t == 0 || has1) softmax_group(sm, a, tmem, t, hf, b, h, qb0 + t, t ? l1 : l0, abort_flag);
+        if (t == 0 || has1) softmax_group<D>(sm, a, tmem, t, hf, b, h, qb0 + t, t ? l1 : l0, abort_flag);
     }
     tc_fence_before_sync();
     __syncthreads();
@@ -518,6 +553,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after_sync();
         tmem_dealloc(tmem, kTmemCols);
     }
+}
+
+template <int D>
+cudaError_t run(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const AttnArgs& a, int64_t grid,
+                cudaStream_t st) {
+    constexpr size_t smem = smem_bytes<D>();
+    static_assert(smem <= 232448, "shared memory per CTA");
+    cudaError_t e = cudaFuncSetAttribute(attention_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    attention_kernel<D><<<static_cast<unsigned>(grid), kThreads, smem, st>>>(tq, tk, tv, a);
+    return cudaGetLastError();
 }
 
 }  // namespace
@@ -539,12 +586,9 @@ cudaError_t launch_attention(const CUtensorMap& tq, const CUtensorMap& tk, const
     a.scale_log2 = scale * 1.4426950408889634f;
     a.status = status;
     a.timeout_ns = timeout_ns;
-    cudaError_t e = cudaFuncSetAttribute(attention_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(kSmemBytes));
-    if (e != cudaSuccess) return e;
     const int64_t grid = static_cast<int64_t>(s.B) * s.heads * a.npairs;
-    attention_kernel<<<static_cast<unsigned>(grid), kThreads, kSmemBytes, st>>>(tq, tk, tv, a);
-    return cudaGetLastError();
+    if (s.d == 128) return run<128>(tq, tk, tv, a, grid, st);
+    return run<96>(tq, tk, tv, a, grid, st);
 }
 
 }  // namespace h3a

@@ -57,21 +57,23 @@ EncodeTiledFn g_encode = nullptr;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// Validates a Q/K/V/O descriptor.  Fills `s` on success.
-h3a_status check_desc(const h3a_qkv_desc* d, Shape* s) {
+// Validates a Q/K/V/O descriptor.  Fills `s` on success.  head_dim 96 for
+// every call; the router and attention also take 128 (wide_ok).
+h3a_status check_desc(const h3a_qkv_desc* d, Shape* s, bool wide_ok = false) {
     if (d == nullptr) return H3A_ERR_INVALID_ARG;
-    if (d->head_dim != kHeadDim) return H3A_ERR_UNSUPPORTED;
+    if (d->head_dim != kHeadDim && !(wide_ok && d->head_dim == kHeadDimWide)) return H3A_ERR_UNSUPPORTED;
     if (d->B < 1 || d->N < 1 || d->heads < 1) return H3A_ERR_INVALID_ARG;
     if (d->stride_b < 0 || d->stride_n < 0 || d->stride_h < 0) return H3A_ERR_INVALID_ARG;
     if ((d->stride_b % 8) || (d->stride_n % 8) || (d->stride_h % 8)) return H3A_ERR_INVALID_ARG;
-    if (d->heads > 1 && d->stride_h < kHeadDim) return H3A_ERR_INVALID_ARG;
-    if (d->N > 1 && d->stride_n < kHeadDim) return H3A_ERR_INVALID_ARG;
+    if (d->heads > 1 && d->stride_h < d->head_dim) return H3A_ERR_INVALID_ARG;
+    if (d->N > 1 && d->stride_n < d->head_dim) return H3A_ERR_INVALID_ARG;
     // byte strides must stay within the tensor-map limit (2^40)
     const int64_t lim = (int64_t(1) << 39);
     if (d->stride_b >= lim || d->stride_n >= lim || d->stride_h >= lim) return H3A_ERR_UNSUPPORTED;
     s->B = d->B;
     s->N = d->N;
     s->heads = d->heads;
+    s->d = d->head_dim;
     s->sb = d->stride_b;
     s->sn = d->stride_n;
     s->sh = d->stride_h;
@@ -81,7 +83,7 @@ h3a_status check_desc(const h3a_qkv_desc* d, Shape* s) {
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 size_t pooled_bytes(const Shape& s, int nblk) {
-    return align256(static_cast<size_t>(s.B) * s.heads * nblk * kHeadDim * sizeof(float));
+    return align256(static_cast<size_t>(s.B) * s.heads * nblk * s.d * sizeof(float));
 }
 
 }  // namespace
@@ -95,12 +97,11 @@ cudaError_t make_qkv_tensor_map(CUtensorMap* map, const void* base, const Shape&
             g_encode = reinterpret_cast<EncodeTiledFn>(fn);
     });
     if (g_encode == nullptr) return cudaErrorNotSupported;
-    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(kHeadDim), static_cast<cuuint64_t>(s.heads),
+    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(s.d), static_cast<cuuint64_t>(s.heads),
                                 static_cast<cuuint64_t>(s.N), static_cast<cuuint64_t>(s.B)};
     // byte strides of dims 1..3; a size-1 dim gets a nominal (unused) stride
     auto stride_or = [](int64_t st, int64_t fallback) { return static_cast<cuuint64_t>((st > 0 ? st : fallback) * 2); };
-    const cuuint64_t strides[3] = {stride_or(s.sh, kHeadDim), stride_or(s.sn, kHeadDim),
-                                   stride_or(s.sb, kHeadDim)};
+    const cuuint64_t strides[3] = {stride_or(s.sh, s.d), stride_or(s.sn, s.d), stride_or(s.sb, s.d)};
     const cuuint32_t box[4] = {32, 1, 128, 1};
     const cuuint32_t elem_strides[4] = {1, 1, 1, 1};
     CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
@@ -122,7 +123,7 @@ h3a_status route_setup(const Shape& s, double sparsity, int32_t block, const voi
     if (block != kBlock) return H3A_ERR_UNSUPPORTED;
     if (!(sparsity >= 0.0 && sparsity < 1.0)) return H3A_ERR_INVALID_ARG;
     *nblk = (s.N + kBlock - 1) / kBlock;
-    if (*nblk > route_max_blocks()) return H3A_ERR_UNSUPPORTED;
+    if (*nblk > route_max_blocks(s.d)) return H3A_ERR_UNSUPPORTED;
     if (static_cast<int64_t>(s.B) * s.heads > 65535) return H3A_ERR_UNSUPPORTED;
     const size_t half = pooled_bytes(s, *nblk);
     if (workspace == nullptr || !aligned16(workspace) || ws_bytes < 2 * half) return H3A_ERR_WORKSPACE;
@@ -187,7 +188,7 @@ int64_t h3a_route_k(int64_t nkv, double sparsity) {
 
 h3a_status h3a_route_workspace_size(const h3a_qkv_desc* d, int32_t block, size_t* bytes) {
     Shape s;
-    h3a_status rc = check_desc(d, &s);
+    h3a_status rc = check_desc(d, &s, true);
     if (rc != H3A_OK) return rc;
     if (bytes == nullptr) return H3A_ERR_INVALID_ARG;
     if (block != kBlock) return H3A_ERR_UNSUPPORTED;
@@ -199,7 +200,7 @@ h3a_status h3a_route_workspace_size(const h3a_qkv_desc* d, int32_t block, size_t
 h3a_status h3a_route(const void* q, const void* k, const h3a_qkv_desc* d, double sparsity, int32_t block,
                      int32_t* block_idx, int64_t* k_out, void* workspace, size_t ws_bytes, h3a_stream_t stream) {
     Shape s;
-    h3a_status rc = check_desc(d, &s);
+    h3a_status rc = check_desc(d, &s, true);
     if (rc != H3A_OK) return rc;
     if (block != kBlock) return H3A_ERR_UNSUPPORTED;
     if (!q || !k || !block_idx) return H3A_ERR_INVALID_ARG;
@@ -253,7 +254,7 @@ h3a_status h3a_attention(const void* q, const void* k, const void* v, const h3a_
                          const int32_t* block_idx, int32_t k_blocks, int32_t block, float scale, void* o,
                          h3a_stream_t stream) {
     Shape s;
-    h3a_status rc = check_desc(d, &s);
+    h3a_status rc = check_desc(d, &s, true);
     if (rc != H3A_OK) return rc;
     if (block != kBlock) return H3A_ERR_UNSUPPORTED;
     if (!q || !k || !v || !o) return H3A_ERR_INVALID_ARG;
@@ -266,7 +267,7 @@ h3a_status h3a_attention(const void* q, const void* k, const void* v, const h3a_
     }
     const int64_t grid = static_cast<int64_t>(s.B) * s.heads * ((nblk + 1) / 2);
     if (grid >= (int64_t(1) << 31)) return H3A_ERR_UNSUPPORTED;
-    if (scale == 0.0f) scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(kHeadDim)));
+    if (scale == 0.0f) scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(s.d)));
     int* status = nullptr;
     rc = status_word(&status);
     if (rc != H3A_OK) return rc;
@@ -312,7 +313,7 @@ h3a_status h3a_selftest_mma(const void* a, const void* b, float* s_out, float* r
     int* status = nullptr;
     h3a_status rc = status_word(&status);
     if (rc != H3A_OK) return rc;
-    Shape s{1, 128, 1, 128 * kHeadDim, kHeadDim, kHeadDim};
+    Shape s{1, 128, 1, kHeadDim, 128 * kHeadDim, kHeadDim, kHeadDim};
     CUtensorMap ta, tb;
     cudaError_t e = make_qkv_tensor_map(&ta, a, s);
     if (e == cudaSuccess) e = make_qkv_tensor_map(&tb, b, s);

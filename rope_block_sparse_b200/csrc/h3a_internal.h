@@ -8,7 +8,8 @@
 
 namespace h3a {
 
-constexpr int kHeadDim = 96;
+constexpr int kHeadDim = 96;       // every call
+constexpr int kHeadDimWide = 128;  // the router and attention also take it (SubBlock's head size)
 constexpr int kBlock = 128;
 
 // Status word bits set by kernels (read back by h3a_last_device_error).
@@ -16,6 +17,7 @@ constexpr int kDevTimeout = 1;
 
 struct Shape {
     int B, N, heads;
+    int d;               // head_dim: 96, or 128 (router and attention)
     int64_t sb, sn, sh;  // element strides; head_dim contiguous
 };
 
@@ -38,7 +40,7 @@ cudaError_t launch_route(const void* q, const void* k, const Shape& s, int nblk,
 cudaError_t launch_route_scores(const float* pooled_q, const float* pooled_k, const Shape& s, int nblk, int kk,
                                 int32_t* idx, cudaStream_t st);
 // Largest nblk the score/top-k kernel supports (shared-memory bound).
-int route_max_blocks();
+int route_max_blocks(int d);
 
 // Attention (attention.cu).  blocks == nullptr: dense.
 cudaError_t launch_attention(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, void* o,

@@ -22,9 +22,10 @@
 namespace h3a {
 namespace {
 
-constexpr int kPoolThreads = 224;    // 672 16-byte vectors per 56-head token row, 3 per thread
+constexpr int kPoolThreads = 224;    // 672 16-byte vectors per CTA row: 56 heads of 96 or 42 of 128
 constexpr int kVecPerThread = 3;
-constexpr int kHeadsPerPoolCta = kPoolThreads * kVecPerThread / (kHeadDim / 8);  // 56
+template <int D>
+constexpr int heads_per_pool_cta() { return kPoolThreads * kVecPerThread / (D / 8); }
 constexpr int kScoreThreads = 512;   // 16 warps
 constexpr int kRowsPerCta = 16;      // query blocks per score CTA (one warp each)
 constexpr int kScoreSmemLimit = 200 * 1024;
@@ -47,16 +48,20 @@ __device__ __forceinline__ void acc8(float* acc, uint4 v) {
     acc[7] += __uint_as_float(v.w & 0xFFFF0000u);
 }
 
-// grid: (nblk, B, 2 tensors x head chunks of 56).  Thread t covers 16-byte
-// vectors t, t+224, t+448 of the chunk's part of a token row (vector v = head
-// 56*chunk + v/12, channels 8*(v%12) .. +7).
+// grid: (nblk, B, 2 tensors x head chunks).  Thread t covers 16-byte vectors
+// t, t+224, t+448 of the chunk's part of a token row (vector v = head
+// HC*chunk + v/(D/8), channels 8*(v%(D/8)) .. +7, HC = 56 heads at D = 96,
+// 42 at D = 128).
+template <int D>
 __global__ void __launch_bounds__(kPoolThreads) block_pool_kernel(const PoolArgs a) {
+    constexpr int kHeadsPerPoolCta = heads_per_pool_cta<D>();
+    constexpr int kVecPerHead = D / 8;
     const int blk = blockIdx.x, b = blockIdx.y, which = blockIdx.z & 1, chunk = blockIdx.z >> 1;
     const __nv_bfloat16* x = a.x[which];
     const int n0 = blk * kBlock;
     const int n1 = min(a.N, n0 + kBlock);
     const int h_base = chunk * kHeadsPerPoolCta;
-    const int vec_per_row = min(kHeadsPerPoolCta, a.heads - h_base) * (kHeadDim / 8);
+    const int vec_per_row = min(kHeadsPerPoolCta, a.heads - h_base) * kVecPerHead;
 
     int64_t off[kVecPerThread];
     bool act[kVecPerThread];
@@ -64,7 +69,7 @@ __global__ void __launch_bounds__(kPoolThreads) block_pool_kernel(const PoolArgs
     for (int u = 0; u < kVecPerThread; ++u) {
         const int v = threadIdx.x + u * kPoolThreads;
         act[u] = v < vec_per_row;
-        const int h = h_base + v / (kHeadDim / 8), c = (v % (kHeadDim / 8)) * 8;
+        const int h = h_base + v / kVecPerHead, c = (v % kVecPerHead) * 8;
         off[u] = static_cast<int64_t>(b) * a.sb + static_cast<int64_t>(h) * a.sh + c;
     }
     float acc[kVecPerThread][8];
@@ -97,8 +102,8 @@ __global__ void __launch_bounds__(kPoolThreads) block_pool_kernel(const PoolArgs
     for (int u = 0; u < kVecPerThread; ++u) {
         if (!act[u]) continue;
         const int v = threadIdx.x + u * kPoolThreads;
-        const int h = h_base + v / (kHeadDim / 8), c = (v % (kHeadDim / 8)) * 8;
-        float* dst = a.out[which] + ((static_cast<int64_t>(b) * a.heads + h) * a.nblk + blk) * kHeadDim + c;
+        const int h = h_base + v / kVecPerHead, c = (v % kVecPerHead) * 8;
+        float* dst = a.out[which] + ((static_cast<int64_t>(b) * a.heads + h) * a.nblk + blk) * D + c;
         float4 lo = make_float4(acc[u][0] * inv_len, acc[u][1] * inv_len, acc[u][2] * inv_len, acc[u][3] * inv_len);
         float4 hi = make_float4(acc[u][4] * inv_len, acc[u][5] * inv_len, acc[u][6] * inv_len, acc[u][7] * inv_len);
         reinterpret_cast<float4*>(dst)[0] = lo;
@@ -122,20 +127,21 @@ __device__ __forceinline__ uint32_t order_key(float f) {
 
 // grid: (ceil(nblk / 16), B*heads).  Dynamic shared memory:
 // qbar[16][96] fp32, scores[16][nblk] fp32, histograms[16][256] u32.
+template <int D>
 __global__ void __launch_bounds__(kScoreThreads) score_topk_kernel(const ScoreArgs a) {
     extern __shared__ __align__(16) float smem[];
     float* qbar = smem;                                   // [16][96]
-    float* scores = qbar + kRowsPerCta * kHeadDim;        // [16][nblk]
+    float* scores = qbar + kRowsPerCta * D;               // [16][nblk]
     uint32_t* hist = reinterpret_cast<uint32_t*>(scores + kRowsPerCta * a.nblk);  // [16][256]
 
     const int bh = blockIdx.y;
     const int i0 = blockIdx.x * kRowsPerCta;
     const int rows = min(kRowsPerCta, a.nblk - i0);
-    const float* qsrc = a.qp + (static_cast<int64_t>(bh) * a.nblk + i0) * kHeadDim;
-    const float* ksrc = a.kp + static_cast<int64_t>(bh) * a.nblk * kHeadDim;
+    const float* qsrc = a.qp + (static_cast<int64_t>(bh) * a.nblk + i0) * D;
+    const float* ksrc = a.kp + static_cast<int64_t>(bh) * a.nblk * D;
 
-    for (int e = threadIdx.x; e < kRowsPerCta * kHeadDim; e += kScoreThreads)
-        qbar[e] = (e < rows * kHeadDim) ? qsrc[e] : 0.f;
+    for (int e = threadIdx.x; e < kRowsPerCta * D; e += kScoreThreads)
+        qbar[e] = (e < rows * D) ? qsrc[e] : 0.f;
     __syncthreads();
 
     // scores[r][j] = (qbar_r . kbar_j) * inv_sqrt_d, dot in channel order
@@ -143,13 +149,13 @@ __global__ void __launch_bounds__(kScoreThreads) score_topk_kernel(const ScoreAr
         float dot[kRowsPerCta];
 #pragma unroll
         for (int r = 0; r < kRowsPerCta; ++r) dot[r] = 0.f;
-        const float4* kj = reinterpret_cast<const float4*>(ksrc + static_cast<int64_t>(j) * kHeadDim);
+        const float4* kj = reinterpret_cast<const float4*>(ksrc + static_cast<int64_t>(j) * D);
 #pragma unroll 4
-        for (int c4 = 0; c4 < kHeadDim / 4; ++c4) {
+        for (int c4 = 0; c4 < D / 4; ++c4) {
             const float4 kv = __ldg(kj + c4);
 #pragma unroll
             for (int r = 0; r < kRowsPerCta; ++r) {
-                const float4 qv = reinterpret_cast<const float4*>(qbar + r * kHeadDim)[c4];
+                const float4 qv = reinterpret_cast<const float4*>(qbar + r * D)[c4];
                 dot[r] = fmaf(qv.x, kv.x, dot[r]);
                 dot[r] = fmaf(qv.y, kv.y, dot[r]);
                 dot[r] = fmaf(qv.z, kv.z, dot[r]);
@@ -238,37 +244,32 @@ __global__ void __launch_bounds__(kScoreThreads) score_topk_kernel(const ScoreAr
     }
 }
 
-size_t score_smem_bytes(int nblk) {
-    return (static_cast<size_t>(kRowsPerCta) * kHeadDim + static_cast<size_t>(kRowsPerCta) * nblk) * sizeof(float) +
+size_t score_smem_bytes(int nblk, int d) {
+    return (static_cast<size_t>(kRowsPerCta) * d + static_cast<size_t>(kRowsPerCta) * nblk) * sizeof(float) +
            static_cast<size_t>(kRowsPerCta) * 256 * sizeof(uint32_t);
 }
 
-}  // namespace
-
-int route_max_blocks() {
-    // largest nblk whose score tile fits the shared-memory budget
-    return static_cast<int>((kScoreSmemLimit - score_smem_bytes(0)) / (kRowsPerCta * sizeof(float)));
-}
-
-cudaError_t launch_route_scores(const float* pooled_q, const float* pooled_k, const Shape& s, int nblk, int kk,
-                                int32_t* idx, cudaStream_t st) {
+template <int D>
+cudaError_t scores(const float* pooled_q, const float* pooled_k, const Shape& s, int nblk, int kk, int32_t* idx,
+                   cudaStream_t st) {
     ScoreArgs a;
     a.qp = pooled_q;
     a.kp = pooled_k;
     a.idx = idx;
     a.nblk = nblk;
     a.kk = kk;
-    a.inv_sqrt_d = static_cast<float>(1.0 / std::sqrt(static_cast<double>(kHeadDim)));
-    const size_t smem = score_smem_bytes(nblk);
-    cudaError_t e =
-        cudaFuncSetAttribute(score_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    a.inv_sqrt_d = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
+    const size_t smem = score_smem_bytes(nblk, D);
+    cudaError_t e = cudaFuncSetAttribute(score_topk_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    score_topk_kernel<<<dim3((nblk + kRowsPerCta - 1) / kRowsPerCta, s.B * s.heads), kScoreThreads, smem, st>>>(a);
+    score_topk_kernel<D><<<dim3((nblk + kRowsPerCta - 1) / kRowsPerCta, s.B * s.heads), kScoreThreads, smem, st>>>(a);
     return cudaGetLastError();
 }
 
-cudaError_t launch_route(const void* q, const void* k, const Shape& s, int nblk, int kk, float* pooled_q,
-                         float* pooled_k, int32_t* idx, cudaStream_t st) {
+template <int D>
+cudaError_t pool(const void* q, const void* k, const Shape& s, int nblk, float* pooled_q, float* pooled_k,
+                 cudaStream_t st) {
     PoolArgs p;
     p.x[0] = static_cast<const __nv_bfloat16*>(q);
     p.x[1] = static_cast<const __nv_bfloat16*>(k);
@@ -280,9 +281,29 @@ cudaError_t launch_route(const void* q, const void* k, const Shape& s, int nblk,
     p.sb = s.sb;
     p.sn = s.sn;
     p.sh = s.sh;
-    const int chunks = (s.heads + kHeadsPerPoolCta - 1) / kHeadsPerPoolCta;
-    block_pool_kernel<<<dim3(nblk, s.B, 2 * chunks), kPoolThreads, 0, st>>>(p);
-    cudaError_t e = cudaGetLastError();
+    constexpr int hc = heads_per_pool_cta<D>();
+    const int chunks = (s.heads + hc - 1) / hc;
+    block_pool_kernel<D><<<dim3(nblk, s.B, 2 * chunks), kPoolThreads, 0, st>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+int route_max_blocks(int d) {
+    // largest nblk whose score tile fits the shared-memory budget
+    return static_cast<int>((kScoreSmemLimit - score_smem_bytes(0, d)) / (kRowsPerCta * sizeof(float)));
+}
+
+cudaError_t launch_route_scores(const float* pooled_q, const float* pooled_k, const Shape& s, int nblk, int kk,
+                                int32_t* idx, cudaStream_t st) {
+    if (s.d == kHeadDimWide) return scores<kHeadDimWide>(pooled_q, pooled_k, s, nblk, kk, idx, st);
+    return scores<kHeadDim>(pooled_q, pooled_k, s, nblk, kk, idx, st);
+}
+
+cudaError_t launch_route(const void* q, const void* k, const Shape& s, int nblk, int kk, float* pooled_q,
+                         float* pooled_k, int32_t* idx, cudaStream_t st) {
+    cudaError_t e = s.d == kHeadDimWide ? pool<kHeadDimWide>(q, k, s, nblk, pooled_q, pooled_k, st)
+                                        : pool<kHeadDim>(q, k, s, nblk, pooled_q, pooled_k, st);
     if (e != cudaSuccess) return e;
     return launch_route_scores(pooled_q, pooled_k, s, nblk, kk, idx, st);
 }

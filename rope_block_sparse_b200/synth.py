@@ -40,6 +40,7 @@ class Workload:
     dist: str
     sparsity: float | None  # None = dense attention
     also_dense: bool = False
+    head_dim: int = HEAD_DIM
 
     @property
     def N(self) -> int:
@@ -60,6 +61,10 @@ WORKLOADS = {
     "video10s": Workload("video10s", 1, 56, (61, 48, 84), "structured", 0.80, also_dense=True),
     # a 16x32x64 = 32,768-token clip for profiler captures: Q, K, V still exceed L2 (352 MB each).
     "clip32k": Workload("clip32k", 1, 56, (16, 32, 64), "structured", 0.75),
+    # the 5 s clip at SubBlock's stated head size: the same 5376-wide hidden state as
+    # 42 heads x 128, block-sparse at 0.75 (router and attention only: the 3D RoPE
+    # layout is defined for 96 channels).
+    "video5s_d128": Workload("video5s_d128", 1, 42, (31, 48, 84), "structured", 0.75, head_dim=128),
 }
 
 _STREAM = {"q": 1, "k": 2, "v": 3, "gamma_q": 4, "gamma_k": 5}
@@ -130,7 +135,7 @@ def draw(B: int, heads: int, grid, dist: str = "normal", seed: int = 0, head_dim
 
 def draw_workload(name: str, seed: int = 0, names=("q", "k", "v")) -> dict:
     w = WORKLOADS[name]
-    return draw(w.B, w.heads, w.grid, w.dist, seed, names=names)
+    return draw(w.B, w.heads, w.grid, w.dist, seed, head_dim=w.head_dim, names=names)
 
 
 def sample_rows(B: int, heads: int, N: int, count: int, seed: int = 1234) -> torch.Tensor:

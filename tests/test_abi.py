@@ -61,7 +61,11 @@ def test_workspace_size():
     nblk = 977
     assert n.value == 2 * ((56 * nblk * 96 * 4 + 255) // 256 * 256)
     assert lib.h3a_route_workspace_size(ctypes.byref(d), 64, ctypes.byref(n)) == 2  # block must be 128
-    bad = _desc(D=128)
+    # 42 heads x 128 (the same 5376-wide hidden state): the router takes head_dim 128
+    wide = _desc(N=124992, heads=42, D=128)
+    assert lib.h3a_route_workspace_size(ctypes.byref(wide), 128, ctypes.byref(n)) == 0
+    assert n.value == 2 * ((42 * nblk * 128 * 4 + 255) // 256 * 256)
+    bad = _desc(D=64)
     assert lib.h3a_route_workspace_size(ctypes.byref(bad), 128, ctypes.byref(n)) == 2
 
 
@@ -91,6 +95,7 @@ def test_prologue_validation():
     assert call(theta=0.0) == 1
     bad = _desc(D=64)
     assert call(d=ctypes.byref(bad)) == 2               # head_dim != 96
+    assert call(d=ctypes.byref(_desc(D=128))) == 2     # the prologue is defined for 96 channels
     odd = h3a.QkvDesc(1, 8064, 56, 96, 8064 * 56 * 96, 56 * 96 + 4, 96)
     assert call(d=ctypes.byref(odd)) == 1               # stride not a multiple of 8 elements
     assert lib.h3a_qk_norm_rope(GOOD, GOOD, None, GOOD, GOOD, grid, 1e4, 1e-6, GOOD, GOOD, None) == 1
@@ -166,8 +171,10 @@ def test_attention_validation():
     assert call(blocks=GOOD, kb=64) == 1              # nblk = 63
     assert call(scale=-1.0) == 1
     assert call(scale=float("inf")) == 1
-    bad = _desc(D=128)
-    assert call(desc=bad) == 2
+    assert call(desc=_desc(D=64)) == 2
+    wide = _desc(N=8064, heads=42, D=128)                # head_dim 128 passes the shape check
+    assert call(desc=wide, o=None) == 1
+    assert call(desc=wide, block=64) == 2
 
 
 def test_python_binding_refuses_cpu_tensors():

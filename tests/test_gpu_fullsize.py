@@ -100,3 +100,28 @@ def test_video5s_fused_prologue_pool_route(orc):
         check_prologue(bits(out[0, torch.as_tensor(tok).cuda()]), want, "video5s fused prologue")
     ora_idx, ora_sc = orc.route(bits(qo), bits(ko), 0.75)
     check_router(idx.cpu().numpy(), ora_idx, ora_sc, "video5s pooled router")
+
+
+def test_video5s_d128_dense_and_sparse(orc):
+    """The 124,992-token clip at head_dim 128 (42 heads), as bench.py runs it with
+    --workload video5s_d128: router on every row, dense and sparse (0.75)
+    attention on 4096 sampled rows; inputs go to the router as drawn."""
+    w = synth.WORKLOADS["video5s_d128"]
+    d = synth.draw_workload("video5s_d128")
+    q, k, v = (d[n].cuda() for n in "qkv")
+    idx = h3a.route(q, k, 0.75)
+    torch.cuda.synchronize()
+    ora_idx, ora_sc = orc.route(d["q"], d["k"], 0.75)
+    check_router(idx.cpu().numpy(), ora_idx, ora_sc, "video5s_d128 router")
+    del ora_sc
+    rows = synth.sample_rows(w.B, w.heads, w.N, SAMPLE).numpy()
+    o = h3a.attention(q, k, v, torch.from_numpy(ora_idx).cuda())
+    torch.cuda.synchronize()
+    assert h3a.last_device_error() == 0
+    check_attention(gather_rows(o, rows), orc.attention_rows(d["q"], d["k"], d["v"], rows, ora_idx),
+                    "video5s_d128 sparse")
+    o = h3a.attention(q, k, v)
+    torch.cuda.synchronize()
+    assert h3a.last_device_error() == 0
+    check_attention(gather_rows(o, rows[:2048]), orc.attention_rows(d["q"], d["k"], d["v"], rows[:2048]),
+                    "video5s_d128 dense")
