@@ -68,6 +68,10 @@ def _load():
         lib.oracle_route.restype = i64
         lib.oracle_attention_rows.argtypes = [P, P, P, i32, i64, i32, i32, P, i64, i32, f64, P, i64, P, i32]
         lib.oracle_attention_rows.restype = i32
+        lib.oracle_residual_adaln.argtypes = [P, P, P, P, P, i32, i64, i32, f64, P, P, i32]
+        lib.oracle_residual_adaln.restype = i32
+        lib.oracle_swiglu.argtypes = [P, i64, i32, P, i32]
+        lib.oracle_swiglu.restype = i32
         assert lib.oracle_abi_version() == 1
         _lib = lib
     return _lib
@@ -245,4 +249,42 @@ def attention_rows(q, k, v, rows, block_idx: np.ndarray | None = None, block: in
                                        _ptr(r), r.size, _ptr(out), nthreads)
     if rc != 0:
         raise ValueError("oracle_attention_rows: bad sizes")
+    return out
+
+
+def residual_adaln(x, f, gate: np.ndarray, shift: np.ndarray, scale: np.ndarray, eps: float = 1e-6,
+                   nthreads: int = 0):
+    """Gated residual + AdaLN update of bf16 [B, R, C] rows (f None: the AdaLN update alone).
+
+    gate, shift, scale: fp32 [B, C].  Returns (h bf16 bits [B, R, C], y fp64 [B, R, C])."""
+    xb = _bits(x)
+    B, R, C = xb.shape
+    fb = None if f is None else _bits(f)
+    if fb is not None and fb.shape != xb.shape:
+        raise ValueError("x and f must have the same shape")
+    g = np.ascontiguousarray(gate if gate is not None else np.zeros((B, C)), dtype=np.float32)
+    sh = np.ascontiguousarray(shift, dtype=np.float32)
+    sc = np.ascontiguousarray(scale, dtype=np.float32)
+    for a in (g, sh, sc):
+        if a.shape != (B, C):
+            raise ValueError("gate, shift, scale must be [B, C]")
+    h = np.empty(xb.shape, dtype=np.uint16)
+    y = np.empty(xb.shape, dtype=np.float64)
+    rc = _load().oracle_residual_adaln(_ptr(xb), None if fb is None else _ptr(fb), _ptr(g), _ptr(sh), _ptr(sc),
+                                       B, R, C, eps, _ptr(h), _ptr(y), nthreads)
+    if rc != 0:
+        raise ValueError("oracle_residual_adaln: bad sizes")
+    return h, y
+
+
+def swiglu(x, nthreads: int = 0) -> np.ndarray:
+    """silu(a) * b for bf16 [R, 2F] rows with halves a | b -> fp64 [R, F]."""
+    xb = _bits(x)
+    R, F2 = xb.shape
+    if F2 % 2:
+        raise ValueError("last dimension must be even (a | b halves)")
+    out = np.empty((R, F2 // 2), dtype=np.float64)
+    rc = _load().oracle_swiglu(_ptr(xb), R, F2 // 2, _ptr(out), nthreads)
+    if rc != 0:
+        raise ValueError("oracle_swiglu: bad sizes")
     return out

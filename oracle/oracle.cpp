@@ -18,6 +18,11 @@
 //   * Dense lossless attention (cocoloop page, opening quote: "no
 //     approximation") and block-sparse attention over the routed KV blocks,
 //     bidirectional (cocoloop page, "Ein paar Grenzen": non-causal).
+//   * The other operators the fused-operator paragraph of the cocoloop page
+//     names -- the AdaLN update, the gated residual path and the SwiGLU
+//     activation -- with their usual DiT definitions (the page gives none):
+//     h = x + gate * f, y = LayerNorm(h) * (1 + scale) + shift with no affine
+//     LayerNorm, and silu(a) * b.
 //
 // Everything is computed in double precision from the bf16 input bits, with
 // plain loops and no blocking, fusion or reordering beyond the definitions.
@@ -375,6 +380,59 @@ int oracle_attention_rows(const uint16_t* q, const uint16_t* k, const uint16_t* 
             for (int c = 0; c < d; ++c) acc[c] += p * bf16_to_double(v[bshd_index(b, keys[t], h, c, N, heads, d)]);
         }
         for (int c = 0; c < d; ++c) out[i * d + c] = acc[c] / denom;
+    });
+    return 0;
+}
+
+// Gated residual followed by the AdaLN update, per token row of width C
+// (cocoloop page, fused-operator paragraph: the AdaLN update and the gated
+// residual path; definitions as in DiT blocks).  For batch b and row r:
+//   h = x + gate[b] * f                 (f == NULL: h = x, the AdaLN update alone)
+//   h is rounded once to bf16 (that is the tensor the block passes on)
+//   mu = mean(h), var = mean((h - mu)^2) over the C channels of the rounded h
+//   y = (h - mu) / sqrt(var + eps) * (1 + scale[b]) + shift[b]
+// x, f: bf16 [B, R, C]; gate, shift, scale: fp32 [B, C].  h_bits receives
+// the rounded h (bf16 bits), y the fp64 result before its rounding.
+int oracle_residual_adaln(const uint16_t* x, const uint16_t* f, const float* gate, const float* shift,
+                          const float* scale, int B, int64_t R, int C, double eps, uint16_t* h_bits, double* y,
+                          int nthreads) {
+    if (B < 1 || R < 0 || C < 1 || eps < 0) return 1;
+    parallel_for(static_cast<int64_t>(B) * R, nthreads, [&](int64_t br) {
+        const int b = static_cast<int>(br / R);
+        const int64_t base = br * C;
+        std::vector<double> h(C);
+        for (int c = 0; c < C; ++c) {
+            double v = bf16_to_double(x[base + c]);
+            if (f) v += static_cast<double>(gate[static_cast<int64_t>(b) * C + c]) * bf16_to_double(f[base + c]);
+            h_bits[base + c] = double_to_bf16_rne(v);
+            h[c] = bf16_to_double(h_bits[base + c]);
+        }
+        double mu = 0.0;
+        for (int c = 0; c < C; ++c) mu += h[c];
+        mu /= C;
+        double var = 0.0;
+        for (int c = 0; c < C; ++c) var += (h[c] - mu) * (h[c] - mu);
+        var /= C;
+        const double rstd = 1.0 / std::sqrt(var + eps);
+        for (int c = 0; c < C; ++c) {
+            const int64_t bc = static_cast<int64_t>(b) * C + c;
+            y[base + c] = (h[c] - mu) * rstd * (1.0 + static_cast<double>(scale[bc])) + static_cast<double>(shift[bc]);
+        }
+    });
+    return 0;
+}
+
+// SwiGLU activation (cocoloop page, fused-operator paragraph): for each row of
+// a bf16 [R, 2F] tensor whose halves are a = [0, F) and b = [F, 2F),
+// out = silu(a) * b = a / (1 + exp(-a)) * b, in fp64.
+int oracle_swiglu(const uint16_t* in, int64_t R, int F, double* out, int nthreads) {
+    if (R < 0 || F < 1) return 1;
+    parallel_for(R, nthreads, [&](int64_t r) {
+        for (int i = 0; i < F; ++i) {
+            const double a = bf16_to_double(in[r * 2 * F + i]);
+            const double bv = bf16_to_double(in[r * 2 * F + F + i]);
+            out[r * F + i] = a / (1.0 + std::exp(-a)) * bv;
+        }
     });
     return 0;
 }

@@ -455,3 +455,105 @@ def test_prologue_variants_agree(orc):
     sub = orc.qk_norm_rope_tokens(x, g, grid, toks)
     np.testing.assert_array_equal(sub, full.reshape(60, 3, D)[toks])
     np.testing.assert_array_equal(orc.qk_norm_rope_bf16(x, g, grid), orc.round_bf16(full))
+
+
+# ---------------------------------------------------------------- gated residual + AdaLN, SwiGLU
+
+def _zeros(B, C):
+    return np.zeros((B, C), dtype=np.float32)
+
+
+def test_adaln_hand_example(orc):
+    """C = 2, x = [1, 3], eps = 0: mean 2, variance 1, so LayerNorm gives [-1, 1];
+    with scale [0.5, 0] and shift [0, 10] the update gives [-1.5, 11]."""
+    x = _bf16([[[1.0, 3.0]]])
+    h, y = orc.residual_adaln(x, None, None, np.array([[0.0, 10.0]], np.float32),
+                              np.array([[0.5, 0.0]], np.float32), eps=0.0)
+    assert np.array_equal(h, x.view(torch.int16).numpy().view(np.uint16))
+    assert np.allclose(y, [[[-1.5, 11.0]]], rtol=0, atol=1e-15)
+
+
+def test_adaln_normalises_rows(orc):
+    """No residual, scale = shift = 0: every row has mean 0 and mean square
+    var / (var + eps) (closed form of the normalisation)."""
+    x = torch.randn(2, 5, 96, generator=torch.Generator().manual_seed(3)).to(torch.bfloat16)
+    eps = 1e-2
+    h, y = orc.residual_adaln(x, None, None, _zeros(2, 96), _zeros(2, 96), eps=eps)
+    xd = x.double().numpy()
+    var = xd.var(axis=-1)
+    assert np.allclose(y.mean(axis=-1), 0.0, atol=1e-13)
+    assert np.allclose((y ** 2).mean(axis=-1), var / (var + eps), rtol=1e-12)
+
+
+def test_adaln_modulation_is_affine_per_channel(orc):
+    """y(scale, shift) = y(0, 0) * (1 + scale) + shift, channel by channel and per batch."""
+    g = torch.Generator().manual_seed(4)
+    x = torch.randn(2, 3, 40, generator=g).to(torch.bfloat16)
+    sc = torch.randn(2, 40, generator=g).numpy().astype(np.float32)
+    sh = torch.randn(2, 40, generator=g).numpy().astype(np.float32)
+    _, y0 = orc.residual_adaln(x, None, None, _zeros(2, 40), _zeros(2, 40))
+    _, y = orc.residual_adaln(x, None, None, sh, sc)
+    want = y0 * (1.0 + sc.astype(np.float64))[:, None, :] + sh.astype(np.float64)[:, None, :]
+    assert np.allclose(y, want, rtol=0, atol=1e-12)
+
+
+def test_adaln_ignores_a_constant_offset(orc):
+    """LayerNorm removes the row mean: adding 4 to every channel of integer-valued
+    rows (exact in bf16) leaves y unchanged."""
+    x = torch.randint(-8, 9, (1, 4, 32), generator=torch.Generator().manual_seed(5)).to(torch.bfloat16)
+    sh = np.linspace(-1, 1, 32, dtype=np.float32)[None]
+    sc = np.linspace(0, 2, 32, dtype=np.float32)[None]
+    _, y0 = orc.residual_adaln(x, None, None, sh, sc)
+    _, y1 = orc.residual_adaln(x + 4, None, None, sh, sc)
+    assert np.allclose(y0, y1, rtol=0, atol=1e-13)
+
+
+def test_gated_residual_terms(orc):
+    """h = x + gate * f: gate 0 gives x bit for bit; x = [1, 1], f = [1, -1] and
+    gate [2, 2] give [3, -1]; f = x with gate 1 doubles x exactly."""
+    g = torch.Generator().manual_seed(6)
+    x = torch.randn(2, 3, 16, generator=g).to(torch.bfloat16)
+    f = torch.randn(2, 3, 16, generator=g).to(torch.bfloat16)
+    xbits = x.view(torch.int16).numpy().view(np.uint16)
+    h, _ = orc.residual_adaln(x, f, _zeros(2, 16), _zeros(2, 16), _zeros(2, 16))
+    assert np.array_equal(h, xbits)
+    h, _ = orc.residual_adaln(x, x, np.ones((2, 16), np.float32), _zeros(2, 16), _zeros(2, 16))
+    assert np.array_equal(h, (x * 2).view(torch.int16).numpy().view(np.uint16))
+    h, _ = orc.residual_adaln(_bf16([[[1.0, 1.0]]]), _bf16([[[1.0, -1.0]]]), np.full((1, 2), 2.0, np.float32),
+                              _zeros(1, 2), _zeros(1, 2))
+    assert np.array_equal(h, _bf16([[[3.0, -1.0]]]).view(torch.int16).numpy().view(np.uint16))
+
+
+def test_gated_residual_gate_is_per_batch(orc):
+    """The gate of batch b scales only batch b's branch."""
+    x = torch.zeros(2, 1, 8).to(torch.bfloat16)
+    f = torch.ones(2, 1, 8).to(torch.bfloat16)
+    gate = np.stack([np.full(8, 0.5), np.full(8, -2.0)]).astype(np.float32)
+    h, _ = orc.residual_adaln(x, f, gate, _zeros(2, 8), _zeros(2, 8))
+    got = torch.from_numpy(h.view(np.int16)).view(torch.bfloat16).float().numpy()
+    assert np.array_equal(got[0], np.full((1, 8), 0.5)) and np.array_equal(got[1], np.full((1, 8), -2.0))
+
+
+def test_swiglu_identities(orc):
+    """silu(a) - silu(-a) = a for any a (sigma(a) + sigma(-a) = 1), silu(0) = 0,
+    silu(a) -> a for large a and -> 0 for very negative a, b = 0 gives 0;
+    the first half of a row is the gated input a, the second half b."""
+    a = np.array([0.75, 1.5, 3.0, -2.25, 0.0, 40.0, -40.0], np.float32)
+    row = np.concatenate([a, -a, np.ones(7, np.float32), np.ones(7, np.float32)])[None]
+    out = orc.swiglu(_bf16(row))[0]
+    ab = _bf16(a).double().numpy()
+    assert np.allclose(out[:7] - out[7:], ab, rtol=0, atol=1e-14)
+    assert out[4] == 0.0
+    assert abs(out[5] - 40.0) < 1e-15 * 40 + 1e-14 and abs(out[12]) < 1e-15
+    zero_b = np.concatenate([a, np.zeros(7, np.float32)])[None]
+    assert np.all(orc.swiglu(_bf16(zero_b)) == 0.0)
+
+
+def test_swiglu_scales_linearly_in_b(orc):
+    """out(a, c * b) = c * out(a, b) for a power-of-two c (exact scaling)."""
+    g = torch.Generator().manual_seed(7)
+    a = torch.randn(3, 10, generator=g)
+    b = torch.randn(3, 10, generator=g)
+    o1 = orc.swiglu(torch.cat([a, b], 1).to(torch.bfloat16))
+    o2 = orc.swiglu(torch.cat([a, 4 * b], 1).to(torch.bfloat16))
+    assert np.allclose(o2, 4 * o1, rtol=1e-15, atol=0)
