@@ -267,6 +267,7 @@ def run_gpu(args, rank, world, local):
         if e is not None:
             e[2].record(stream)
     torch.cuda.synchronize()
+    dit = time_dit_ops(h3a, synth, q, k, B, N, heads * w.head_dim, stream, world, rank)
     if wide:
         kern_ms["prologue"] = kern_ms["prologue_pool"] = 0.0
         kern_ms["router"] = kern_ms["router_scores"]
@@ -379,7 +380,7 @@ def run_gpu(args, rank, world, local):
             "attention_dense": {"ms": round(kern_ms["attention_dense"], 3), "TFLOP/s": round(dense_tflops, 2)},
             "sparse_speedup_incl_router": round(kern_ms["attention_dense"] /
                                                 (kern_ms["attention_sparse"] + route_cost), 3),
-        },
+        } | {name: dict(ent, frac_hbm=round(ent["GB/s"] / pk["hbm_gbs"], 4)) for name, ent in dit.items()},
         "gpu_launches": args.steps * 4,
         "clocks": clocks,
         "e2e": e2e,
@@ -387,6 +388,47 @@ def run_gpu(args, rank, world, local):
     if args.cpu_baseline and world == 1:
         line["cpu_baseline"] = cpu_baseline(d, w, args.cpu_rows)
     return line
+
+
+def time_dit_ops(h3a, synth, q, k, B, N, width, stream, world, rank, reps=10):
+    """The other fused DiT operators at the clip's shape, outside the timed step:
+    the gated residual + AdaLN update over B*N rows of the `width`-wide hidden
+    state (x and f are the resident Q and K buffers viewed as [B, N, width]) and
+    SwiGLU at an FFN width of 4 * width (the [a | b] input drawn on the device
+    from a seeded generator).  Algorithmic bytes: 8 per element (x, f read; h, y
+    written) and 6 per SwiGLU output (a, b read; out written)."""
+    x = q.view(B, N, width)
+    f = k.view(B, N, width)
+    cond = synth.draw_dit(B, 1, width, seed=rank)
+    gate, shift, scale = (cond[n].to(q.device) for n in ("gate", "shift", "scale"))
+    h, y = torch.empty_like(x), torch.empty_like(x)
+    ffn = 4 * width
+    g = torch.Generator(device=q.device).manual_seed(1000 + rank)
+    a_b = torch.randn((B * N, 2 * ffn), generator=g, device=q.device, dtype=torch.float32).to(torch.bfloat16)
+    out = torch.empty((B * N, ffn), dtype=torch.bfloat16, device=q.device)
+
+    def t(fn):
+        for _ in range(3):
+            fn()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return allreduce_max(e0.elapsed_time(e1) / reps, world)
+
+    ms_ad = t(lambda: h3a.residual_adaln(x, f, gate, shift, scale, out=(h, y)))
+    ms_sw = t(lambda: h3a.swiglu(a_b, out=out))
+    del a_b, out, h, y
+    torch.cuda.empty_cache()
+    rows = B * N
+    return {
+        "dit_residual_adaln_untimed_step": {"ms": round(ms_ad, 4), "rows": rows, "width": width,
+                                            "GB/s": round(8.0 * rows * width / (ms_ad * 1e-3) / 1e9, 1)},
+        "dit_swiglu_untimed_step": {"ms": round(ms_sw, 4), "rows": rows, "ffn_width": ffn,
+                                    "GB/s": round(6.0 * rows * ffn / (ms_sw * 1e-3) / 1e9, 1)},
+    }
 
 
 # ----------------------------------------------------------------- oracle (CPU)

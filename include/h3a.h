@@ -140,6 +140,38 @@ h3a_status h3a_route_pooled(const h3a_qkv_desc* d, double sparsity, int32_t bloc
                             int32_t* block_idx, int64_t* k_out, const void* workspace,
                             size_t ws_bytes, h3a_stream_t stream);
 
+/* Gated residual followed by the AdaLN update, one pass over device memory.
+ * Source: news.cocoloop.cn MiniMax-H3 SGLang report, section "Erst drei
+ * übereinandergelegte Beschleunigungsebenen", fused-operator paragraph (the
+ * AdaLN update and the gated residual path fused like QK-RMSNorm + 3D RoPE,
+ * no result changed); the page gives no formulas, these are the DiT block's.
+ * For batch b and token row r of width C:
+ *   h = x + gate[b] * f, rounded once to bf16 (f == NULL: h = x)
+ *   y = (h - mean(h)) / sqrt(var(h) + eps) * (1 + scale[b]) + shift[b]
+ *   (LayerNorm without affine, statistics over the C channels of the rounded
+ *   h, fp32 arithmetic, y rounded once to bf16).
+ * x, f        : device bf16 [B, rows, width], contiguous; f may be NULL.
+ * gate, shift, scale: device fp32 [B, width] (gate only read when f != NULL).
+ * h_out       : device bf16 [B, rows, width], written when f != NULL (then
+ *               required; may equal x); ignored when f == NULL.
+ * y_out       : device bf16 [B, rows, width]; must not overlap x, f or h_out.
+ * All pointers 16-byte aligned.
+ * Errors: INVALID_ARG for null/misaligned pointers, width not a positive
+ * multiple of 8, eps < 0; UNSUPPORTED for width > 14336 or B*rows >= 2^31. */
+h3a_status h3a_residual_adaln(const void* x, const void* f, const float* gate, const float* shift,
+                              const float* scale, int32_t B, int64_t rows, int32_t width, float eps,
+                              void* h_out, void* y_out, h3a_stream_t stream);
+
+/* SwiGLU activation: out = silu(a) * b = a / (1 + exp(-a)) * b.
+ * Source: the same fused-operator paragraph (the SwiGLU activation).
+ * in  : device bf16 [rows, 2 * ffn_width], contiguous; each row is a (the
+ *       first ffn_width channels) followed by b.
+ * out : device bf16 [rows, ffn_width], contiguous; must not overlap in.
+ * fp32 arithmetic, one rounding to bf16.  Both pointers 16-byte aligned.
+ * Errors: INVALID_ARG for null/misaligned pointers or ffn_width not a
+ * positive multiple of 8. */
+h3a_status h3a_swiglu(const void* in, int64_t rows, int32_t ffn_width, void* out, h3a_stream_t stream);
+
 /* Capacity of the scratch built into h3a_route_noalloc: 64 MiB, enough for
  * B * heads * ceil(N / 128) <= 87,381 (e.g. 56 heads of a 124,992-token clip). */
 #define H3A_ROUTE_NOALLOC_MAX_BYTES ((size_t)64 << 20)

@@ -22,7 +22,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libh3a.so")
-SOURCES = ["h3a_api.cu", "prologue.cu", "router.cu", "attention.cu", "selftest.cu", "route_noalloc.cu"]
+SOURCES = ["h3a_api.cu", "prologue.cu", "router.cu", "attention.cu", "selftest.cu", "route_noalloc.cu", "dit_ops.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O2", "--expt-relaxed-constexpr",
          "-Xptxas", "-v", "-I", INCLUDE, "-I", CSRC]

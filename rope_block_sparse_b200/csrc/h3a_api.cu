@@ -281,6 +281,31 @@ h3a_status h3a_attention(const void* q, const void* k, const void* v, const h3a_
     return e == cudaSuccess ? H3A_OK : cuda_fail(e);
 }
 
+h3a_status h3a_residual_adaln(const void* x, const void* f, const float* gate, const float* shift,
+                              const float* scale, int32_t B, int64_t rows, int32_t width, float eps, void* h_out,
+                              void* y_out, h3a_stream_t stream) {
+    if (B < 1 || rows < 0 || width < 8) return H3A_ERR_INVALID_ARG;
+    if (width % 8) return H3A_ERR_INVALID_ARG;
+    if (width > residual_adaln_max_width()) return H3A_ERR_UNSUPPORTED;
+    if (static_cast<int64_t>(B) * rows >= (int64_t(1) << 31)) return H3A_ERR_UNSUPPORTED;
+    if (!x || !shift || !scale || !y_out) return H3A_ERR_INVALID_ARG;
+    if (f && (!gate || !h_out)) return H3A_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(shift) || !aligned16(scale) || !aligned16(y_out)) return H3A_ERR_INVALID_ARG;
+    if ((f && !aligned16(f)) || (gate && !aligned16(gate)) || (h_out && !aligned16(h_out)))
+        return H3A_ERR_INVALID_ARG;
+    if (!(eps >= 0.0f)) return H3A_ERR_INVALID_ARG;
+    cudaError_t e = launch_residual_adaln(x, f, f ? gate : nullptr, shift, scale, B, rows, width, eps,
+                                          f ? h_out : nullptr, y_out, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? H3A_OK : cuda_fail(e);
+}
+
+h3a_status h3a_swiglu(const void* in, int64_t rows, int32_t ffn_width, void* out, h3a_stream_t stream) {
+    if (rows < 0 || ffn_width < 8 || (ffn_width % 8)) return H3A_ERR_INVALID_ARG;
+    if (!in || !out || !aligned16(in) || !aligned16(out)) return H3A_ERR_INVALID_ARG;
+    cudaError_t e = launch_swiglu(in, rows, ffn_width, out, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? H3A_OK : cuda_fail(e);
+}
+
 h3a_status h3a_last_device_error(h3a_stream_t stream) {
     int* status = nullptr;
     h3a_status rc = status_word(&status);

@@ -47,6 +47,13 @@ cudaError_t launch_attention(const CUtensorMap& tq, const CUtensorMap& tk, const
                              const Shape& s, const int32_t* blocks, int k_blocks, float scale, int* status,
                              uint64_t timeout_ns, cudaStream_t st);
 
+// Gated residual + AdaLN update and SwiGLU (dit_ops.cu).
+cudaError_t launch_residual_adaln(const void* x, const void* f, const float* gate, const float* shift,
+                                  const float* scale, int B, int64_t rows, int width, float eps, void* h_out,
+                                  void* y_out, cudaStream_t st);
+int residual_adaln_max_width();
+cudaError_t launch_swiglu(const void* in, int64_t rows, int ffn_width, void* out, cudaStream_t st);
+
 // Self-checks (selftest.cu).
 cudaError_t launch_selftest_wait(uint64_t limit_ns, int* status, cudaStream_t st);
 cudaError_t launch_selftest_exp2(const float* x, float* y, int n, int poly, cudaStream_t st);

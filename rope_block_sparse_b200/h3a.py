@@ -26,7 +26,7 @@ STATUS_NAMES = {0: "H3A_OK", 1: "H3A_ERR_INVALID_ARG", 2: "H3A_ERR_UNSUPPORTED",
 EXPORTS = ("h3a_qk_norm_rope", "h3a_route_k", "h3a_route_workspace_size", "h3a_route", "h3a_attention",
            "h3a_status_string", "h3a_last_cuda_error_string", "h3a_last_device_error",
            "h3a_selftest_wait_timeout", "h3a_selftest_mma", "h3a_selftest_exp2", "h3a_route_noalloc",
-           "h3a_qk_norm_rope_pool", "h3a_route_pooled")
+           "h3a_qk_norm_rope_pool", "h3a_route_pooled", "h3a_residual_adaln", "h3a_swiglu")
 ROUTE_NOALLOC_MAX_BYTES = 64 << 20  # H3A_ROUTE_NOALLOC_MAX_BYTES
 
 
@@ -94,6 +94,10 @@ def load() -> ctypes.CDLL:
     lib.h3a_route_pooled.argtypes = [ctypes.POINTER(QkvDesc), f64, i32, P, ctypes.POINTER(ctypes.c_int64), P,
                                      ctypes.c_size_t, P]
     lib.h3a_route_pooled.restype = st
+    lib.h3a_residual_adaln.argtypes = [P, P, P, P, P, i32, i64, i32, f32, P, P, P]
+    lib.h3a_residual_adaln.restype = st
+    lib.h3a_swiglu.argtypes = [P, i64, i32, P, P]
+    lib.h3a_swiglu.restype = st
     _lib = lib
     return lib
 
@@ -267,6 +271,44 @@ def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block_idx: torc
     d = desc_of(q)
     _check("h3a_attention", lib.h3a_attention(_ptr(q), _ptr(k), _ptr(v), ctypes.byref(d), _ptr(block_idx), kb,
                                               block, float(scale), _ptr(out), _stream_handle()))
+    return out
+
+
+def residual_adaln(x: torch.Tensor, f: torch.Tensor | None, gate: torch.Tensor | None, shift: torch.Tensor,
+                   scale: torch.Tensor, eps: float = 1e-6, out=None):
+    """Gated residual + AdaLN update of bf16 [B, rows, C] rows: h = x + gate*f (bf16),
+    y = LayerNorm(h) * (1 + scale) + shift.  gate/shift/scale: fp32 [B, C].
+    f None: the AdaLN update of x alone.  Returns (h or None, y); out=(h, y) writes in place."""
+    lib = load()
+    if x.dim() != 3 or not x.is_cuda or x.dtype != torch.bfloat16 or not x.is_contiguous():
+        raise ValueError("x must be a contiguous bf16 [B, rows, C] CUDA tensor")
+    B, R, C = x.shape
+    for t in ([f] if f is not None else []):
+        if t.shape != x.shape or t.dtype != torch.bfloat16 or not t.is_contiguous() or not t.is_cuda:
+            raise ValueError("f must match x")
+    for name, t in (("shift", shift), ("scale", scale)) + ((("gate", gate),) if f is not None else ()):
+        if t is None or t.shape != (B, C) or t.dtype != torch.float32 or not t.is_contiguous() or not t.is_cuda:
+            raise ValueError(f"{name} must be a contiguous fp32 [B, C] CUDA tensor")
+    if out is not None:
+        h, y = out
+    else:
+        h = torch.empty_like(x) if f is not None else None
+        y = torch.empty_like(x)
+    _check("h3a_residual_adaln", lib.h3a_residual_adaln(_ptr(x), _ptr(f), _ptr(gate if f is not None else None),
+                                                        _ptr(shift), _ptr(scale), B, R, C, float(eps), _ptr(h),
+                                                        _ptr(y), _stream_handle()))
+    return h, y
+
+
+def swiglu(x: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
+    """silu(a) * b for bf16 [rows, 2F] rows laid out [a | b] -> bf16 [rows, F]."""
+    lib = load()
+    if x.dim() != 2 or not x.is_cuda or x.dtype != torch.bfloat16 or not x.is_contiguous() or x.shape[1] % 2:
+        raise ValueError("x must be a contiguous bf16 [rows, 2F] CUDA tensor")
+    R, F = x.shape[0], x.shape[1] // 2
+    if out is None:
+        out = torch.empty((R, F), dtype=torch.bfloat16, device=x.device)
+    _check("h3a_swiglu", lib.h3a_swiglu(_ptr(x), R, F, _ptr(out), _stream_handle()))
     return out
 
 

@@ -67,7 +67,8 @@ WORKLOADS = {
     "video5s_d128": Workload("video5s_d128", 1, 42, (31, 48, 84), "structured", 0.75, head_dim=128),
 }
 
-_STREAM = {"q": 1, "k": 2, "v": 3, "gamma_q": 4, "gamma_k": 5}
+_STREAM = {"q": 1, "k": 2, "v": 3, "gamma_q": 4, "gamma_k": 5,
+           "x": 11, "f": 12, "gate": 13, "shift": 14, "scale": 15, "ffn": 16}
 
 
 def _gen(seed: int, name: str) -> torch.Generator:
@@ -144,3 +145,31 @@ def sample_rows(B: int, heads: int, N: int, count: int, seed: int = 1234) -> tor
     count = min(count, total)
     g = torch.Generator().manual_seed(seed)
     return torch.randperm(total, generator=g)[:count].sort().values
+
+
+def draw_dit(B: int, rows: int, width: int, ffn_width: int = 0, seed: int = 0) -> dict:
+    """Inputs of the gated residual + AdaLN update and of SwiGLU, on the CPU.
+
+    x (residual stream) and f (branch output): bf16 [B, rows, width] ~ N(0, 1);
+    gate, shift, scale (per-batch conditioning, as a timestep embedding gives):
+    fp32 [B, width] ~ 0.5 * N(0, 1); with ffn_width > 0 also ffn: bf16
+    [B * rows, 2 * ffn_width] ~ N(0, 1), the [a | b] input of SwiGLU.  Generated
+    a batch at a time from one generator per tensor."""
+    out = {}
+    for name in ("x", "f"):
+        g = _gen(seed, name)
+        t = torch.empty((B, rows, width), dtype=torch.bfloat16)
+        for b in range(B):
+            t[b] = torch.randn((rows, width), generator=g).to(torch.bfloat16)
+        out[name] = t
+    for name in ("gate", "shift", "scale"):
+        out[name] = (0.5 * torch.randn((B, width), generator=_gen(seed, name))).to(torch.float32)
+    if ffn_width > 0:
+        g = _gen(seed, "ffn")
+        t = torch.empty((B * rows, 2 * ffn_width), dtype=torch.bfloat16)
+        step = max(1, (1 << 24) // (2 * ffn_width))
+        for r0 in range(0, B * rows, step):
+            r1 = min(B * rows, r0 + step)
+            t[r0:r1] = torch.randn((r1 - r0, 2 * ffn_width), generator=g).to(torch.bfloat16)
+        out["ffn"] = t
+    return out

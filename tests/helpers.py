@@ -101,3 +101,24 @@ def gather_rows(o: torch.Tensor, rows: np.ndarray) -> np.ndarray:
     bh, n = r // N, r % N
     b, h = bh // H, bh % H
     return o[b.to(o.device), n.to(o.device), h.to(o.device)].double().cpu().numpy()
+
+
+def check_fp32_rounding(gpu_bits: np.ndarray, want_bits: np.ndarray, label: str = "", floor: int = 3):
+    """The prologue rule for outputs computed in fp32 and rounded once to bf16,
+    sized for small cases: every output within one bf16 ulp (or 2^-18 near
+    zero) of the oracle's correctly rounded value, and at most
+    max(0.1% of the outputs, `floor`) of them not equal to it.  fp32 arithmetic
+    (an approximate rsqrt, another summation order) moves a result across a
+    bf16 rounding boundary with a probability of about 1e-4 per output, so on a
+    few hundred outputs "99.9% exact" would forbid even one such crossing."""
+    assert gpu_bits.shape == want_bits.shape
+    inexact = int(np.sum(gpu_bits != want_bits))
+    allowed = max(int(0.001 * gpu_bits.size), floor)
+    assert inexact <= allowed, f"{label}: {inexact} of {gpu_bits.size} outputs not correctly rounded (> {allowed})"
+    ulps = np.abs(bf16_order(gpu_bits) - bf16_order(want_bits))
+    far = ulps > 1
+    if far.any():
+        worst = float(np.max(np.abs(bits_to_f64(gpu_bits[far]) - bits_to_f64(want_bits[far]))))
+        assert worst <= PROLOGUE_ABS_FLOOR, (
+            f"{label}: {int(far.sum())} outputs beyond 1 ulp, worst absolute error {worst:.3g}")
+    return inexact

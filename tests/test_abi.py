@@ -177,6 +177,28 @@ def test_attention_validation():
     assert call(desc=wide, block=64) == 2
 
 
+@NO_GPU
+def test_dit_ops_validation():
+    lib = h3a.load()
+
+    def ad(x=GOOD, f=GOOD, gate=GOOD, h=GOOD, y=GOOD, B=1, R=4, C=5376, eps=1e-6):
+        return lib.h3a_residual_adaln(x, f, gate, GOOD, GOOD, B, R, C, eps, h, y, None)
+
+    assert ad(C=12) == 1                    # not a multiple of 8
+    assert ad(C=0) == 1
+    assert ad(C=14336 + 8) == 2             # wider than a CTA's registers hold
+    assert ad(x=None) == 1
+    assert ad(gate=None) == 1               # a residual needs its gate
+    assert ad(h=None) == 1                  # ... and an h output
+    assert ad(y=MISALIGNED) == 1
+    assert ad(eps=-1.0) == 1
+    assert ad(B=0) == 1
+    assert lib.h3a_swiglu(GOOD, 4, 12, GOOD, None) == 1
+    assert lib.h3a_swiglu(None, 4, 16, GOOD, None) == 1
+    assert lib.h3a_swiglu(GOOD, 4, 16, MISALIGNED, None) == 1
+    assert lib.h3a_swiglu(GOOD, -1, 16, GOOD, None) == 1
+
+
 def test_python_binding_refuses_cpu_tensors():
     q = torch.zeros(1, 128, 2, 96, dtype=torch.bfloat16)
     with pytest.raises(ValueError, match="CUDA"):
