@@ -72,6 +72,8 @@ def _load():
         lib.oracle_residual_adaln.restype = i32
         lib.oracle_swiglu.argtypes = [P, i64, i32, P, i32]
         lib.oracle_swiglu.restype = i32
+        lib.oracle_residual_diff.argtypes = [P, P, i64]
+        lib.oracle_residual_diff.restype = f64
         assert lib.oracle_abi_version() == 1
         _lib = lib
     return _lib
@@ -288,3 +290,11 @@ def swiglu(x, nthreads: int = 0) -> np.ndarray:
     if rc != 0:
         raise ValueError("oracle_swiglu: bad sizes")
     return out
+
+
+def residual_diff(cur, prev) -> float:
+    """Relative L1 difference sum|cur - prev| / sum|prev| of two bf16 tensors (fp64)."""
+    a, b = _bits(cur).reshape(-1), _bits(prev).reshape(-1)
+    if a.size != b.size:
+        raise ValueError("cur and prev must have the same number of elements")
+    return float(_load().oracle_residual_diff(_ptr(np.ascontiguousarray(a)), _ptr(np.ascontiguousarray(b)), a.size))

@@ -23,6 +23,10 @@
 //     activation -- with their usual DiT definitions (the page gives none):
 //     h = x + gate * f, y = LayerNorm(h) * (1 + scale) + shift with no affine
 //     LayerNorm, and silu(a) * b.
+//   * The Cache-DiT reuse decision (same page, the paragraph after it): a
+//     residual-difference threshold, 0.04 conservative or 0.08 in stride mode,
+//     decides whether a step's result is reused; read as the relative L1
+//     difference sum|cur - prev| / sum|prev| of two steps' residuals.
 //
 // Everything is computed in double precision from the bf16 input bits, with
 // plain loops and no blocking, fusion or reordering beyond the definitions.
@@ -435,6 +439,24 @@ int oracle_swiglu(const uint16_t* in, int64_t R, int F, double* out, int nthread
         }
     });
     return 0;
+}
+
+// Cache-DiT reuse decision quantity (cocoloop page, Cache-DiT paragraph: a
+// residual-difference threshold of 0.04 / 0.08 decides reuse between
+// adjacent denoising steps): the relative L1 difference of the current
+// step's residual to the previous step's,
+//   rel = sum_i |cur_i - prev_i| / sum_i |prev_i|   (fp64; +inf if prev is 0
+//   everywhere and cur is not, 0 if both are),
+// over n bf16 values.  Reuse when rel < threshold.
+double oracle_residual_diff(const uint16_t* cur, const uint16_t* prev, int64_t n) {
+    double num = 0.0, den = 0.0;
+    for (int64_t i = 0; i < n; ++i) {
+        const double a = bf16_to_double(cur[i]), b = bf16_to_double(prev[i]);
+        num += std::fabs(a - b);
+        den += std::fabs(b);
+    }
+    if (den == 0.0) return num == 0.0 ? 0.0 : INFINITY;
+    return num / den;
 }
 
 }  // extern "C"

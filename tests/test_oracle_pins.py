@@ -557,3 +557,33 @@ def test_swiglu_scales_linearly_in_b(orc):
     o1 = orc.swiglu(torch.cat([a, b], 1).to(torch.bfloat16))
     o2 = orc.swiglu(torch.cat([a, 4 * b], 1).to(torch.bfloat16))
     assert np.allclose(o2, 4 * o1, rtol=1e-15, atol=0)
+
+
+# ---------------------------------------------------------------- Cache-DiT residual difference
+
+def test_residual_diff_closed_forms(orc):
+    """Equal tensors give 0; prev = 2 * cur gives |cur - 2cur| / |2cur| = 1/2 exactly;
+    cur = 0 gives 1; cur = -prev gives 2; prev is the base (cur = 2 * prev gives 1,
+    not 1/2); all-zero inputs give 0 and a zero base with a nonzero cur gives inf."""
+    g = torch.Generator().manual_seed(8)
+    b = torch.randn(1000, generator=g).to(torch.bfloat16)
+    assert orc.residual_diff(b, b) == 0.0
+    assert orc.residual_diff(b, b * 2) == 0.5
+    assert orc.residual_diff(b * 2, b) == 1.0
+    assert orc.residual_diff(torch.zeros_like(b), b) == 1.0
+    assert orc.residual_diff(-b, b) == 2.0
+    z = torch.zeros(16, dtype=torch.bfloat16)
+    assert orc.residual_diff(z, z) == 0.0
+    assert orc.residual_diff(torch.ones(16, dtype=torch.bfloat16), z) == math.inf
+
+
+def test_residual_diff_hand_example_and_scale_invariance(orc):
+    """cur = [1, 2, 3, 4], prev = [1, 1, 4, 2]: |diff| = 0+1+1+2 = 4, |prev| = 8 -> 0.5;
+    scaling both by 2^k leaves it unchanged."""
+    cur, prev = _bf16([1, 2, 3, 4]), _bf16([1, 1, 4, 2])
+    assert orc.residual_diff(cur, prev) == 0.5
+    g = torch.Generator().manual_seed(9)
+    a = torch.randn(777, generator=g).to(torch.bfloat16)
+    c = torch.randn(777, generator=g).to(torch.bfloat16)
+    r = orc.residual_diff(a, c)
+    assert orc.residual_diff(a * 8, c * 8) == pytest.approx(r, rel=1e-15)
