@@ -395,8 +395,9 @@ def time_dit_ops(h3a, synth, q, k, B, N, width, stream, world, rank, reps=10):
     the gated residual + AdaLN update over B*N rows of the `width`-wide hidden
     state (x and f are the resident Q and K buffers viewed as [B, N, width]) and
     SwiGLU at an FFN width of 4 * width (the [a | b] input drawn on the device
-    from a seeded generator).  Algorithmic bytes: 8 per element (x, f read; h, y
-    written) and 6 per SwiGLU output (a, b read; out written)."""
+    from a seeded generator), and the Cache-DiT residual difference of x
+    against f.  Algorithmic bytes: 8 per element (x, f read; h, y written), 6
+    per SwiGLU output (a, b read; out written), 4 per compared value."""
     x = q.view(B, N, width)
     f = k.view(B, N, width)
     cond = synth.draw_dit(B, 1, width, seed=rank)
@@ -420,6 +421,9 @@ def time_dit_ops(h3a, synth, q, k, B, N, width, stream, world, rank, reps=10):
 
     ms_ad = t(lambda: h3a.residual_adaln(x, f, gate, shift, scale, out=(h, y)))
     ms_sw = t(lambda: h3a.swiglu(a_b, out=out))
+    ws = torch.empty(h3a.h3a.RESIDUAL_DIFF_WORKSPACE_BYTES, dtype=torch.uint8, device=q.device)
+    rel = (torch.empty(1, dtype=torch.float64, device=q.device), torch.empty(1, dtype=torch.int32, device=q.device))
+    ms_rd = t(lambda: h3a.residual_diff(x, f, 0.04, workspace=ws, out=rel))
     del a_b, out, h, y
     torch.cuda.empty_cache()
     rows = B * N
@@ -428,6 +432,8 @@ def time_dit_ops(h3a, synth, q, k, B, N, width, stream, world, rank, reps=10):
                                             "GB/s": round(8.0 * rows * width / (ms_ad * 1e-3) / 1e9, 1)},
         "dit_swiglu_untimed_step": {"ms": round(ms_sw, 4), "rows": rows, "ffn_width": ffn,
                                     "GB/s": round(6.0 * rows * ffn / (ms_sw * 1e-3) / 1e9, 1)},
+        "cache_dit_residual_diff_untimed_step": {"ms": round(ms_rd, 4), "values": rows * width,
+                                                 "GB/s": round(4.0 * rows * width / (ms_rd * 1e-3) / 1e9, 1)},
     }
 
 

@@ -172,6 +172,29 @@ h3a_status h3a_residual_adaln(const void* x, const void* f, const float* gate, c
  * positive multiple of 8. */
 h3a_status h3a_swiglu(const void* in, int64_t rows, int32_t ffn_width, void* out, h3a_stream_t stream);
 
+/* Device workspace h3a_residual_diff needs: 32 KB (partial sums). */
+#define H3A_RESIDUAL_DIFF_WORKSPACE_BYTES ((size_t)32768)
+
+/* The Cache-DiT reuse decision between two denoising steps.
+ * Source: news.cocoloop.cn MiniMax-H3 SGLang report, Cache-DiT paragraph
+ * after the fused-operator one (results are reused between adjacent steps
+ * when a residual-difference threshold allows: 0.04 conservative, 0.08 in
+ * stride mode); read as the relative L1 difference
+ *   rel = sum_i |cur_i - prev_i| / sum_i |prev_i|
+ * (0 if both are zero, +inf if only prev is), reuse = rel < threshold.
+ * cur, prev : device bf16 arrays of n values (n a positive multiple of 8),
+ *             16-byte aligned.
+ * workspace : device, >= H3A_RESIDUAL_DIFF_WORKSPACE_BYTES, 16-B aligned.
+ * rel_out   : device fp64 scalar; reuse_out: device int32 scalar or NULL.
+ * Sums: each 8 values in fp32, then fp64 in a fixed order (deterministic);
+ * rel agrees with an fp64 sum to about 1e-7 relative, so a decision can only
+ * differ from an exact one for rel within that band of the threshold.
+ * Errors: INVALID_ARG for null/misaligned pointers, n not a positive multiple
+ * of 8, threshold < 0 or NaN; WORKSPACE if the workspace is null or small. */
+h3a_status h3a_residual_diff(const void* cur, const void* prev, int64_t n, double threshold,
+                             void* workspace, size_t ws_bytes, double* rel_out, int32_t* reuse_out,
+                             h3a_stream_t stream);
+
 /* Capacity of the scratch built into h3a_route_noalloc: 64 MiB, enough for
  * B * heads * ceil(N / 128) <= 87,381 (e.g. 56 heads of a 124,992-token clip). */
 #define H3A_ROUTE_NOALLOC_MAX_BYTES ((size_t)64 << 20)

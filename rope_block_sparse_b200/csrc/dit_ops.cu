@@ -12,14 +12,21 @@
 //                           pass over HBM: x and f read once, h and y written
 //                           once.  f == null gives the AdaLN update alone.
 //   swiglu_kernel           out = silu(a) * b for rows [a | b] of width 2F.
+//   residual_diff_*         the Cache-DiT reuse decision (same page, next
+//                           paragraph: a residual-difference threshold of 0.04
+//                           or 0.08 decides reuse between adjacent denoising
+//                           steps), read as rel = sum|cur - prev| / sum|prev|.
 //
-// Both are HBM-bound.  residual_adaln: one 224-thread CTA per token row, each
+// All are HBM-bound.  residual_adaln: one 224-thread CTA per token row, each
 // thread holding up to VPT 16-byte vectors of the row in registers, so the
 // mean and the variance (exact two-pass, in fp32) need no second read; the
 // two reductions go through warp shuffles and shared memory.  swiglu: a
 // grid-stride loop over 16-byte output vectors, two per iteration.
+// residual_diff: a grid-stride pass writing one fp64 partial pair per CTA to a
+// caller workspace, then one CTA adding them in index order (deterministic).
 #include <cuda_bf16.h>
 
+#include <algorithm>
 #include <cmath>
 
 #include "h3a_internal.h"
@@ -190,6 +197,80 @@ __global__ void __launch_bounds__(256) swiglu_kernel(const SwigluArgs a) {
     }
 }
 
+// Relative L1 difference, stage 1: CTA c writes (sum|cur - prev|, sum|prev|)
+// over its grid-stride share of 16-byte vectors to partial[2c], [2c + 1].
+// Each 8-element vector is summed in fp32 (|a - b| and |b| of bf16 values)
+// and added to fp64 accumulators; the CTA total goes through fp64 shuffles.
+constexpr int kDiffThreads = 256;
+constexpr int kDiffMaxCtas = 2048;
+
+__device__ __forceinline__ double warp_sum_d(double v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+// CTA-wide fp64 sums of (x, y), deterministic; valid in thread 0.
+__device__ __forceinline__ void cta_sum2_d(double& x, double& y) {
+    __shared__ double red[2][kDiffThreads / 32];
+    x = warp_sum_d(x);
+    y = warp_sum_d(y);
+    const int warp = threadIdx.x >> 5;
+    if ((threadIdx.x & 31) == 0) {
+        red[0][warp] = x;
+        red[1][warp] = y;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        x = y = 0.0;
+        for (int w = 0; w < kDiffThreads / 32; ++w) {
+            x += red[0][w];
+            y += red[1][w];
+        }
+    }
+}
+
+__global__ void __launch_bounds__(kDiffThreads) residual_diff_partial_kernel(const uint4* cur, const uint4* prev,
+                                                                             int64_t nvec, double* partial) {
+    double num = 0.0, den = 0.0;
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * kDiffThreads;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * kDiffThreads + threadIdx.x; i < nvec; i += stride) {
+        float a[8], b[8];
+        unpack8(__ldg(cur + i), a);
+        unpack8(__ldg(prev + i), b);
+        float n8 = 0.f, d8 = 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            n8 += fabsf(a[e] - b[e]);
+            d8 += fabsf(b[e]);
+        }
+        num += static_cast<double>(n8);
+        den += static_cast<double>(d8);
+    }
+    cta_sum2_d(num, den);
+    if (threadIdx.x == 0) {
+        partial[2 * blockIdx.x] = num;
+        partial[2 * blockIdx.x + 1] = den;
+    }
+}
+
+// Stage 2: one CTA adds the partials in index order and decides reuse.
+__global__ void __launch_bounds__(kDiffThreads) residual_diff_final_kernel(const double* partial, int nparts,
+                                                                           double threshold, double* rel_out,
+                                                                           int32_t* reuse_out) {
+    double num = 0.0, den = 0.0;
+    for (int p = threadIdx.x; p < nparts; p += kDiffThreads) {
+        num += partial[2 * p];
+        den += partial[2 * p + 1];
+    }
+    cta_sum2_d(num, den);
+    if (threadIdx.x == 0) {
+        const double rel = den == 0.0 ? (num == 0.0 ? 0.0 : INFINITY) : num / den;
+        *rel_out = rel;
+        if (reuse_out) *reuse_out = rel < threshold ? 1 : 0;
+    }
+}
+
 template <int VPT>
 cudaError_t adaln(const AdalnArgs& a, int64_t total_rows, cudaStream_t st) {
     residual_adaln_kernel<VPT><<<static_cast<unsigned>(total_rows), kRowThreads, 0, st>>>(a);
@@ -227,6 +308,26 @@ cudaError_t launch_residual_adaln(const void* x, const void* f, const float* gat
         case 7: return adaln<7>(a, total, st);
         default: return adaln<8>(a, total, st);
     }
+}
+
+size_t residual_diff_workspace_bytes() { return sizeof(double) * 2 * kDiffMaxCtas; }
+
+cudaError_t launch_residual_diff(const void* cur, const void* prev, int64_t n, double threshold, void* workspace,
+                                 double* rel_out, int32_t* reuse_out, cudaStream_t st) {
+    const int64_t nvec = n / 8;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    int64_t ctas = (nvec + 4 * kDiffThreads - 1) / (4 * kDiffThreads);
+    ctas = std::max<int64_t>(1, std::min<int64_t>(ctas, std::min<int64_t>(static_cast<int64_t>(sms) * 8, kDiffMaxCtas)));
+    double* partial = static_cast<double*>(workspace);
+    residual_diff_partial_kernel<<<static_cast<unsigned>(ctas), kDiffThreads, 0, st>>>(
+        static_cast<const uint4*>(cur), static_cast<const uint4*>(prev), nvec, partial);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    residual_diff_final_kernel<<<1, kDiffThreads, 0, st>>>(partial, static_cast<int>(ctas), threshold, rel_out,
+                                                          reuse_out);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_swiglu(const void* in, int64_t rows, int ffn_width, void* out, cudaStream_t st) {

@@ -306,6 +306,20 @@ h3a_status h3a_swiglu(const void* in, int64_t rows, int32_t ffn_width, void* out
     return e == cudaSuccess ? H3A_OK : cuda_fail(e);
 }
 
+h3a_status h3a_residual_diff(const void* cur, const void* prev, int64_t n, double threshold, void* workspace,
+                             size_t ws_bytes, double* rel_out, int32_t* reuse_out, h3a_stream_t stream) {
+    if (n < 8 || (n % 8)) return H3A_ERR_INVALID_ARG;
+    if (!cur || !prev || !rel_out || !aligned16(cur) || !aligned16(prev)) return H3A_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(rel_out) & 7u) || (reinterpret_cast<uintptr_t>(reuse_out) & 3u))
+        return H3A_ERR_INVALID_ARG;
+    if (!(threshold >= 0.0)) return H3A_ERR_INVALID_ARG;
+    if (workspace == nullptr || !aligned16(workspace) || ws_bytes < residual_diff_workspace_bytes())
+        return H3A_ERR_WORKSPACE;
+    cudaError_t e = launch_residual_diff(cur, prev, n, threshold, workspace, rel_out, reuse_out,
+                                         reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? H3A_OK : cuda_fail(e);
+}
+
 h3a_status h3a_last_device_error(h3a_stream_t stream) {
     int* status = nullptr;
     h3a_status rc = status_word(&status);

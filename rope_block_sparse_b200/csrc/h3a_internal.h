@@ -53,6 +53,10 @@ cudaError_t launch_residual_adaln(const void* x, const void* f, const float* gat
                                   void* y_out, cudaStream_t st);
 int residual_adaln_max_width();
 cudaError_t launch_swiglu(const void* in, int64_t rows, int ffn_width, void* out, cudaStream_t st);
+// Cache-DiT residual difference (dit_ops.cu): rel = sum|cur - prev| / sum|prev|.
+size_t residual_diff_workspace_bytes();
+cudaError_t launch_residual_diff(const void* cur, const void* prev, int64_t n, double threshold, void* workspace,
+                                 double* rel_out, int32_t* reuse_out, cudaStream_t st);
 
 // Self-checks (selftest.cu).
 cudaError_t launch_selftest_wait(uint64_t limit_ns, int* status, cudaStream_t st);

@@ -26,8 +26,10 @@ STATUS_NAMES = {0: "H3A_OK", 1: "H3A_ERR_INVALID_ARG", 2: "H3A_ERR_UNSUPPORTED",
 EXPORTS = ("h3a_qk_norm_rope", "h3a_route_k", "h3a_route_workspace_size", "h3a_route", "h3a_attention",
            "h3a_status_string", "h3a_last_cuda_error_string", "h3a_last_device_error",
            "h3a_selftest_wait_timeout", "h3a_selftest_mma", "h3a_selftest_exp2", "h3a_route_noalloc",
-           "h3a_qk_norm_rope_pool", "h3a_route_pooled", "h3a_residual_adaln", "h3a_swiglu")
+           "h3a_qk_norm_rope_pool", "h3a_route_pooled", "h3a_residual_adaln", "h3a_swiglu",
+           "h3a_residual_diff")
 ROUTE_NOALLOC_MAX_BYTES = 64 << 20  # H3A_ROUTE_NOALLOC_MAX_BYTES
+RESIDUAL_DIFF_WORKSPACE_BYTES = 32768  # H3A_RESIDUAL_DIFF_WORKSPACE_BYTES
 
 
 class H3AError(RuntimeError):
@@ -98,6 +100,8 @@ def load() -> ctypes.CDLL:
     lib.h3a_residual_adaln.restype = st
     lib.h3a_swiglu.argtypes = [P, i64, i32, P, P]
     lib.h3a_swiglu.restype = st
+    lib.h3a_residual_diff.argtypes = [P, P, i64, f64, P, ctypes.c_size_t, P, P, P]
+    lib.h3a_residual_diff.restype = st
     _lib = lib
     return lib
 
@@ -310,6 +314,29 @@ def swiglu(x: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
         out = torch.empty((R, F), dtype=torch.bfloat16, device=x.device)
     _check("h3a_swiglu", lib.h3a_swiglu(_ptr(x), R, F, _ptr(out), _stream_handle()))
     return out
+
+
+def residual_diff(cur: torch.Tensor, prev: torch.Tensor, threshold: float = 0.04,
+                  workspace: torch.Tensor | None = None, out=None):
+    """Cache-DiT reuse decision: rel = sum|cur - prev| / sum|prev| over two bf16 tensors of
+    the same size, reuse = rel < threshold.  Returns device tensors (rel fp64 [1], reuse int32 [1])."""
+    lib = load()
+    for t in (cur, prev):
+        if not t.is_cuda or t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise ValueError("cur and prev must be contiguous bf16 CUDA tensors")
+    if cur.numel() != prev.numel():
+        raise ValueError("cur and prev must have the same number of values")
+    if workspace is None:
+        workspace = torch.empty(RESIDUAL_DIFF_WORKSPACE_BYTES, dtype=torch.uint8, device=cur.device)
+    if out is None:
+        rel = torch.empty(1, dtype=torch.float64, device=cur.device)
+        reuse = torch.empty(1, dtype=torch.int32, device=cur.device)
+    else:
+        rel, reuse = out
+    _check("h3a_residual_diff", lib.h3a_residual_diff(_ptr(cur), _ptr(prev), cur.numel(), float(threshold),
+                                                      _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                                      _ptr(rel), _ptr(reuse), _stream_handle()))
+    return rel, reuse
 
 
 def last_device_error() -> int:

@@ -68,7 +68,7 @@ WORKLOADS = {
 }
 
 _STREAM = {"q": 1, "k": 2, "v": 3, "gamma_q": 4, "gamma_k": 5,
-           "x": 11, "f": 12, "gate": 13, "shift": 14, "scale": 15, "ffn": 16}
+           "x": 11, "f": 12, "gate": 13, "shift": 14, "scale": 15, "ffn": 16, "prev": 17, "delta": 18}
 
 
 def _gen(seed: int, name: str) -> torch.Generator:
@@ -173,3 +173,11 @@ def draw_dit(B: int, rows: int, width: int, ffn_width: int = 0, seed: int = 0) -
             t[r0:r1] = torch.randn((r1 - r0, 2 * ffn_width), generator=g).to(torch.bfloat16)
         out["ffn"] = t
     return out
+
+
+def draw_step_pair(n: int, sigma: float, seed: int = 0):
+    """Residuals of two adjacent denoising steps, bf16 [n]: prev ~ N(0, 1) and
+    cur = prev + sigma * N(0, 1), so sum|cur - prev| / sum|prev| is close to sigma."""
+    prev = torch.randn(n, generator=_gen(seed, "prev"))
+    cur = prev + sigma * torch.randn(n, generator=_gen(seed, "delta"))
+    return cur.to(torch.bfloat16), prev.to(torch.bfloat16)

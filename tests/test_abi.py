@@ -198,6 +198,18 @@ def test_dit_ops_validation():
     assert lib.h3a_swiglu(GOOD, 4, 16, MISALIGNED, None) == 1
     assert lib.h3a_swiglu(GOOD, -1, 16, GOOD, None) == 1
 
+    def rd(cur=GOOD, n=4096, thr=0.04, w=GOOD, wsb=32768, rel=GOOD, reuse=GOOD):
+        return lib.h3a_residual_diff(cur, GOOD, n, thr, w, wsb, rel, reuse, None)
+
+    assert rd(n=12) == 1
+    assert rd(n=0) == 1
+    assert rd(cur=None) == 1
+    assert rd(rel=P(0x10004)) == 1          # fp64 output must be 8-byte aligned
+    assert rd(thr=-1.0) == 1
+    assert rd(thr=float("nan")) == 1
+    assert rd(w=None) == 5
+    assert rd(wsb=32767) == 5
+
 
 def test_python_binding_refuses_cpu_tensors():
     q = torch.zeros(1, 128, 2, 96, dtype=torch.bfloat16)

@@ -75,3 +75,50 @@ def test_dit_ops_reject_bad_widths():
         h3a.residual_adaln(x, None, None, v, v)
     with pytest.raises(h3a.H3AError, match="INVALID_ARG"):
         h3a.swiglu(torch.zeros(2, 24, dtype=torch.bfloat16, device="cuda"))
+
+
+# ---------------------------------------------------------------- Cache-DiT residual difference
+
+@pytest.mark.parametrize("n", [8, 8 * 1_000_003, 8064 * 5376])
+def test_residual_diff_matches_oracle(orc, n):
+    cur, prev = synth.draw_step_pair(n, 0.05, seed=n % 97)
+    rel, reuse = h3a.residual_diff(cur.cuda(), prev.cuda(), 0.04)
+    torch.cuda.synchronize()
+    want = orc.residual_diff(cur, prev)
+    got = float(rel.item())
+    assert abs(got - want) <= 1e-6 * want, (got, want)
+    assert int(reuse.item()) == int(want < 0.04) or abs(want - 0.04) <= 1e-6 * 0.04
+
+
+@pytest.mark.parametrize("sigma", [0.02, 0.06, 0.1])
+def test_residual_diff_decisions(orc, sigma):
+    """rel near 0.02 reuses at both page thresholds, near 0.06 only in stride mode
+    (0.08), near 0.1 at neither; the decision is the oracle's rel < threshold."""
+    cur, prev = synth.draw_step_pair(1 << 20, sigma, seed=5)
+    want = orc.residual_diff(cur, prev)
+    for thr in (0.04, 0.08):
+        assert abs(want - thr) > 1e-3
+        rel, reuse = h3a.residual_diff(cur.cuda(), prev.cuda(), thr)
+        torch.cuda.synchronize()
+        assert int(reuse.item()) == int(want < thr)
+
+
+def test_residual_diff_deterministic_and_special_values():
+    cur, prev = synth.draw_step_pair(1 << 22, 0.05, seed=6)
+    c, p = cur.cuda(), prev.cuda()
+    r1, _ = h3a.residual_diff(c, p)
+    r2, _ = h3a.residual_diff(c, p)
+    z = torch.zeros(64, dtype=torch.bfloat16, device="cuda")
+    rz, uz = h3a.residual_diff(z, z)
+    ri, ui = h3a.residual_diff(torch.ones_like(z), z)
+    torch.cuda.synchronize()
+    assert r1.item() == r2.item()
+    assert rz.item() == 0.0 and uz.item() == 1
+    assert ri.item() == float("inf") and ui.item() == 0
+
+
+def test_residual_diff_refuses_small_workspace():
+    z = torch.zeros(64, dtype=torch.bfloat16, device="cuda")
+    small = torch.empty(1024, dtype=torch.uint8, device="cuda")
+    with pytest.raises(h3a.H3AError, match="WORKSPACE"):
+        h3a.residual_diff(z, z, workspace=small)
