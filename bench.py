@@ -32,6 +32,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 WORKLOAD = "video5s_sparse"
+FFN_WIDTH = 14336  # DiT FFN width of the model table (52hbtv.com H3-Image page, section 二)
 SPARSITY = 0.75
 METRIC = "attention TFLOP/s and % of B200 bf16 peak at ~125k tokens; prologue GB/s vs HBM"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -394,8 +395,9 @@ def time_dit_ops(h3a, synth, q, k, B, N, width, stream, world, rank, reps=10):
     """The other fused DiT operators at the clip's shape, outside the timed step:
     the gated residual + AdaLN update over B*N rows of the `width`-wide hidden
     state (x and f are the resident Q and K buffers viewed as [B, N, width]) and
-    SwiGLU at an FFN width of 4 * width (the [a | b] input drawn on the device
-    from a seeded generator), and the Cache-DiT residual difference of x
+    SwiGLU at the model's FFN width of 14,336 (52hbtv.com H3-Image page,
+    section 二, model table; the [a | b] input drawn on the device from a seeded
+    generator), and the Cache-DiT residual difference of x
     against f.  Algorithmic bytes: 8 per element (x, f read; h, y written), 6
     per SwiGLU output (a, b read; out written), 4 per compared value."""
     x = q.view(B, N, width)
@@ -403,7 +405,7 @@ def time_dit_ops(h3a, synth, q, k, B, N, width, stream, world, rank, reps=10):
     cond = synth.draw_dit(B, 1, width, seed=rank)
     gate, shift, scale = (cond[n].to(q.device) for n in ("gate", "shift", "scale"))
     h, y = torch.empty_like(x), torch.empty_like(x)
-    ffn = 4 * width
+    ffn = FFN_WIDTH
     g = torch.Generator(device=q.device).manual_seed(1000 + rank)
     a_b = torch.randn((B * N, 2 * ffn), generator=g, device=q.device, dtype=torch.float32).to(torch.bfloat16)
     out = torch.empty((B * N, ffn), dtype=torch.bfloat16, device=q.device)

@@ -85,6 +85,14 @@ h3a_status h3a_qk_norm_rope(const void* q, const void* k, const h3a_qkv_desc* d,
  * Returns -1 if sparsity is outside [0, 1) or nkv < 1. */
 int64_t h3a_route_k(int64_t nkv, double sparsity);
 
+/* Sparsity to use at a denoising step: the router prunes KV blocks from the
+ * first_sparse_step-th step on (news.cocoloop.cn MiniMax-H3 SGLang report,
+ * SubBlock paragraph: from the 10th step), steps counted from 1.  Returns
+ * `sparsity` when step >= first_sparse_step, 0.0 (dense attention) before,
+ * and -1.0 if step < 1, first_sparse_step < 1 or sparsity is outside [0, 1).
+ * Host only; no device work. */
+double h3a_step_sparsity(int32_t step, int32_t first_sparse_step, double sparsity);
+
 /* Bytes of device workspace h3a_route needs: two fp32 [B, heads, nblk,
  * head_dim] pooled tensors, nblk = ceil(N / block), head_dim 96 or 128.
  * Returns INVALID_ARG/UNSUPPORTED for bad descriptors. */

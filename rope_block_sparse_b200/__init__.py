@@ -16,8 +16,8 @@ arguments.  ``synth`` holds the seeded synthetic input generators.
 """
 from .h3a import (H3AError, attention, attention_core, last_device_error, load, qk_norm_rope, qk_norm_rope_pool,
                   residual_adaln, residual_diff, route, route_k, route_pooled, route_workspace_size, selftest_exp2,
-                  selftest_mma, selftest_wait_timeout, swiglu)
+                  selftest_mma, selftest_wait_timeout, step_sparsity, swiglu)
 
 __all__ = ["H3AError", "attention", "attention_core", "last_device_error", "load", "qk_norm_rope",
            "qk_norm_rope_pool", "residual_adaln", "residual_diff", "route", "route_k", "route_pooled", "route_workspace_size",
-           "selftest_exp2", "selftest_mma", "selftest_wait_timeout", "swiglu"]
+           "selftest_exp2", "selftest_mma", "selftest_wait_timeout", "step_sparsity", "swiglu"]

@@ -178,6 +178,11 @@ h3a_status h3a_qk_norm_rope(const void* q, const void* k, const h3a_qkv_desc* d,
     return e == cudaSuccess ? H3A_OK : cuda_fail(e);
 }
 
+double h3a_step_sparsity(int32_t step, int32_t first_sparse_step, double sparsity) {
+    if (step < 1 || first_sparse_step < 1 || !(sparsity >= 0.0 && sparsity < 1.0)) return -1.0;
+    return step >= first_sparse_step ? sparsity : 0.0;
+}
+
 int64_t h3a_route_k(int64_t nkv, double sparsity) {
     if (nkv < 1 || !(sparsity >= 0.0 && sparsity < 1.0)) return -1;
     int64_t kk = static_cast<int64_t>(std::ceil((1.0 - sparsity) * static_cast<double>(nkv) - 1e-9));

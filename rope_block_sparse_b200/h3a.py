@@ -27,7 +27,7 @@ EXPORTS = ("h3a_qk_norm_rope", "h3a_route_k", "h3a_route_workspace_size", "h3a_r
            "h3a_status_string", "h3a_last_cuda_error_string", "h3a_last_device_error",
            "h3a_selftest_wait_timeout", "h3a_selftest_mma", "h3a_selftest_exp2", "h3a_route_noalloc",
            "h3a_qk_norm_rope_pool", "h3a_route_pooled", "h3a_residual_adaln", "h3a_swiglu",
-           "h3a_residual_diff")
+           "h3a_residual_diff", "h3a_step_sparsity")
 ROUTE_NOALLOC_MAX_BYTES = 64 << 20  # H3A_ROUTE_NOALLOC_MAX_BYTES
 RESIDUAL_DIFF_WORKSPACE_BYTES = 32768  # H3A_RESIDUAL_DIFF_WORKSPACE_BYTES
 
@@ -102,6 +102,8 @@ def load() -> ctypes.CDLL:
     lib.h3a_swiglu.restype = st
     lib.h3a_residual_diff.argtypes = [P, P, i64, f64, P, ctypes.c_size_t, P, P, P]
     lib.h3a_residual_diff.restype = st
+    lib.h3a_step_sparsity.argtypes = [i32, i32, f64]
+    lib.h3a_step_sparsity.restype = f64
     _lib = lib
     return lib
 
@@ -223,6 +225,17 @@ def _route_out(q: torch.Tensor, nblk: int, kk: int, out: torch.Tensor | None) ->
     if out.shape != (B, H, nblk, kk) or out.dtype != torch.int32 or not out.is_contiguous():
         raise ValueError("out must be a contiguous int32 [B, heads, nblk, k] tensor")
     return out
+
+
+FIRST_SPARSE_STEP = 10  # the router works from the 10th denoising step on
+
+
+def step_sparsity(step: int, sparsity: float = 0.75, first_sparse_step: int = FIRST_SPARSE_STEP) -> float:
+    """Sparsity at denoising step `step` (from 1): 0.0 (dense) before first_sparse_step."""
+    s = float(load().h3a_step_sparsity(int(step), int(first_sparse_step), float(sparsity)))
+    if s < 0:
+        raise ValueError(f"bad step schedule: step={step}, first_sparse_step={first_sparse_step}, sparsity={sparsity}")
+    return s
 
 
 def route_k(nkv: int, sparsity: float) -> int:
@@ -372,9 +385,13 @@ def selftest_exp2(x: torch.Tensor, use_poly: bool = True) -> torch.Tensor:
 
 def attention_core(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, gamma_q: torch.Tensor,
                    gamma_k: torch.Tensor, grid, sparsity: float | None = None, theta: float = 10000.0,
-                   eps: float = 1e-6, workspace: torch.Tensor | None = None):
+                   eps: float = 1e-6, workspace: torch.Tensor | None = None, step: int | None = None):
     """The whole per-layer core: prologue over Q/K, then dense attention
-    (sparsity None) or router + block-sparse attention.  Returns (o, block_idx or None)."""
+    (sparsity None) or router + block-sparse attention.  With `step` (denoising
+    step, from 1) the sparsity applies only from step 10 on, dense before.
+    Returns (o, block_idx or None)."""
+    if sparsity is not None and step is not None:
+        sparsity = step_sparsity(step, sparsity) or None
     if sparsity is None:
         qn, kn = qk_norm_rope(q, k, gamma_q, gamma_k, grid, theta, eps)
         return attention(qn, kn, v), None

@@ -211,6 +211,23 @@ def test_dit_ops_validation():
     assert rd(wsb=32767) == 5
 
 
+def test_step_schedule_follows_the_page():
+    """The router works from the 10th denoising step on (tests/golden/page_facts.txt):
+    steps 1..9 dense, 10 onward at the given sparsity; bad arguments give -1."""
+    lib = h3a.load()
+    facts = open(os.path.join(ROOT, "tests", "golden", "page_facts.txt")).read().split()
+    first = int(facts[facts.index("subblock_first_sparse_step") + 1])
+    assert first == h3a.FIRST_SPARSE_STEP == 10
+    for step in range(1, first):
+        assert lib.h3a_step_sparsity(step, first, 0.75) == 0.0
+    for step in (first, first + 1, 50):
+        assert lib.h3a_step_sparsity(step, first, 0.8) == 0.8
+    assert lib.h3a_step_sparsity(0, first, 0.75) == -1.0
+    assert lib.h3a_step_sparsity(5, 0, 0.75) == -1.0
+    assert lib.h3a_step_sparsity(12, first, 1.0) == -1.0
+    assert h3a.step_sparsity(9) == 0.0 and h3a.step_sparsity(10) == 0.75
+
+
 def test_python_binding_refuses_cpu_tensors():
     q = torch.zeros(1, 128, 2, 96, dtype=torch.bfloat16)
     with pytest.raises(ValueError, match="CUDA"):

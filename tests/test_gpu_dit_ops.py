@@ -57,7 +57,8 @@ def test_residual_adaln_in_place_matches():
     assert torch.equal(y2.view(torch.int16), y.view(torch.int16))
 
 
-SWIGLU_CASES = [("small", 33, 1344), ("min_width", 5, 8), ("ffn_4x", 7, 21504)]
+# the model's FFN width is 14,336 (52hbtv.com H3-Image page, section 二, model table)
+SWIGLU_CASES = [("small", 33, 1344), ("min_width", 5, 8), ("h3_ffn", 7, 14336), ("wide", 3, 21504)]
 
 
 @pytest.mark.parametrize("name,R,F", SWIGLU_CASES, ids=[c[0] for c in SWIGLU_CASES])

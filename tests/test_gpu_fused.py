@@ -122,3 +122,22 @@ def test_fused_workspace_too_small_is_refused():
         h3a.qk_norm_rope_pool(q, k, d["gamma_q"].cuda(), d["gamma_k"].cuda(), grid, workspace=small)
     with pytest.raises(h3a.H3AError, match="WORKSPACE"):
         h3a.route_pooled(q, 0.5, small)
+
+
+def test_attention_core_follows_the_step_schedule():
+    """attention_core with a denoising step: dense (no block lists) before step 10,
+    the routed sparse path from step 10 on -- each equal, bit for bit, to the
+    calls it stands for."""
+    grid, heads = (4, 16, 40), 3                   # 2560 tokens, 20 blocks
+    d = synth.draw(1, heads, grid, "structured", 4)
+    q, k, v = d["q"].cuda(), d["k"].cuda(), d["v"].cuda()
+    gq, gk = d["gamma_q"].cuda(), d["gamma_k"].cuda()
+    o9, b9 = h3a.attention_core(q, k, v, gq, gk, grid, sparsity=0.75, step=9)
+    o10, b10 = h3a.attention_core(q, k, v, gq, gk, grid, sparsity=0.75, step=10)
+    qn, kn = h3a.qk_norm_rope(q, k, gq, gk, grid)
+    dense = h3a.attention(qn, kn, v)
+    blocks = h3a.route(qn, kn, 0.75)
+    sparse = h3a.attention(qn, kn, v, blocks)
+    torch.cuda.synchronize()
+    assert b9 is None and torch.equal(o9, dense)
+    assert torch.equal(b10, blocks) and torch.equal(o10, sparse)
