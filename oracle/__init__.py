@@ -74,6 +74,8 @@ def _load():
         lib.oracle_swiglu.restype = i32
         lib.oracle_residual_diff.argtypes = [P, P, i64]
         lib.oracle_residual_diff.restype = f64
+        lib.oracle_qk_fullnorm_rope_bf16.argtypes = [P, i32, i64, i32, i32, P, i32, i32, i32, f64, f64, P, i32]
+        lib.oracle_qk_fullnorm_rope_bf16.restype = i32
         assert lib.oracle_abi_version() == 1
         _lib = lib
     return _lib
@@ -298,3 +300,20 @@ def residual_diff(cur, prev) -> float:
     if a.size != b.size:
         raise ValueError("cur and prev must have the same number of elements")
     return float(_load().oracle_residual_diff(_ptr(np.ascontiguousarray(a)), _ptr(np.ascontiguousarray(b)), a.size))
+
+
+def qk_fullnorm_rope_bf16(x, gamma: np.ndarray, grid, theta: float = 10000.0, eps: float = 1e-6,
+                          nthreads: int = 0) -> np.ndarray:
+    """The prologue with the RMSNorm over the token's whole hidden state (all heads;
+    gamma fp32 [heads * d]), then per-head 3D RoPE, rounded to bf16 -> uint16 bits."""
+    xb = _bits(x)
+    B, N, heads, d = xb.shape
+    g = np.ascontiguousarray(gamma, dtype=np.float32).reshape(-1)
+    if g.size != heads * d:
+        raise ValueError("gamma must have heads * d entries")
+    out = np.empty(xb.shape, dtype=np.uint16)
+    rc = _load().oracle_qk_fullnorm_rope_bf16(_ptr(xb), B, N, heads, d, _ptr(g), grid[0], grid[1], grid[2], theta,
+                                              eps, _ptr(out), nthreads)
+    if rc != 0:
+        raise ValueError("oracle_qk_fullnorm_rope_bf16: bad sizes")
+    return out

@@ -388,6 +388,41 @@ int oracle_attention_rows(const uint16_t* q, const uint16_t* k, const uint16_t* 
     return 0;
 }
 
+// The prologue with the RMSNorm spanning the token's whole hidden state (all
+// heads, heads * d channels, one gain per hidden channel) instead of each
+// head: the other reading of "QK-RMSNorm" in the cocoloop page's fused-operator
+// paragraph.  Then the same per-head 3D RoPE, and one rounding to bf16:
+//   r = 1 / sqrt(sum over all heads and channels of x^2 / (heads * d) + eps)
+//   y[h, c] = RoPE_h(x[h, :] * r * gamma[h * d + :])[c]
+// gamma: fp32 [heads * d].  out: bf16 bits, layout of x.
+int oracle_qk_fullnorm_rope_bf16(const uint16_t* x, int B, int64_t N, int heads, int d, const float* gamma,
+                                 int T, int H, int W, double theta, double eps, uint16_t* out, int nthreads) {
+    if (B < 0 || N < 0 || heads <= 0 || d <= 0 || d % 6 != 0) return -1;
+    if (static_cast<int64_t>(T) * H * W != N) return -1;
+    parallel_for(static_cast<int64_t>(B) * N, nthreads, [&](int64_t bn) {
+        const int b = static_cast<int>(bn / N);
+        const int64_t n = bn % N;
+        int pos[3];
+        oracle_token_position(n, T, H, W, pos);
+        double ss = 0.0;
+        for (int h = 0; h < heads; ++h)
+            for (int c = 0; c < d; ++c) {
+                const double v = bf16_to_double(x[bshd_index(b, n, h, c, N, heads, d)]);
+                ss += v * v;
+            }
+        const double r = 1.0 / std::sqrt(ss / (static_cast<double>(heads) * d) + eps);
+        std::vector<double> yv(d);
+        for (int h = 0; h < heads; ++h) {
+            for (int c = 0; c < d; ++c)
+                yv[c] = bf16_to_double(x[bshd_index(b, n, h, c, N, heads, d)]) * r *
+                        static_cast<double>(gamma[h * d + c]);
+            oracle_rope3d(yv.data(), d, pos, theta);
+            for (int c = 0; c < d; ++c) out[bshd_index(b, n, h, c, N, heads, d)] = double_to_bf16_rne(yv[c]);
+        }
+    });
+    return 0;
+}
+
 // Gated residual followed by the AdaLN update, per token row of width C
 // (cocoloop page, fused-operator paragraph: the AdaLN update and the gated
 // residual path; definitions as in DiT blocks).  For batch b and row r:

@@ -587,3 +587,37 @@ def test_residual_diff_hand_example_and_scale_invariance(orc):
     c = torch.randn(777, generator=g).to(torch.bfloat16)
     r = orc.residual_diff(a, c)
     assert orc.residual_diff(a * 8, c * 8) == pytest.approx(r, rel=1e-15)
+
+
+# ---------------------------------------------------------------- full-width QK-RMSNorm
+
+def test_fullnorm_with_one_head_is_the_per_head_prologue(orc):
+    """With a single head the hidden state is the head: the full-width prologue
+    equals the per-head one bit for bit."""
+    g = torch.Generator().manual_seed(10)
+    x = torch.randn(1, 60, 1, D, generator=g).to(torch.bfloat16)
+    gamma = (1 + 0.1 * torch.randn(D, generator=g)).numpy().astype(np.float32)
+    grid = (3, 4, 5)
+    assert np.array_equal(orc.qk_fullnorm_rope_bf16(x, gamma, grid), orc.qk_norm_rope_bf16(x, gamma, grid))
+
+
+def test_fullnorm_couples_the_heads(orc):
+    """At the grid origin (RoPE is the identity) with unit gains: every head of a
+    token is divided by the same RMS over all its heads.  Head 0 = 1 everywhere,
+    head 1 = 3 everywhere: mean square (1 + 9) / 2 = 5, so the outputs are
+    1/sqrt(5) and 3/sqrt(5) (eps 0), where the per-head norm would give 1 and 1."""
+    x = torch.cat([torch.ones(1, 1, 1, D), 3 * torch.ones(1, 1, 1, D)], dim=2).to(torch.bfloat16)
+    out = orc.qk_fullnorm_rope_bf16(x, np.ones(2 * D, np.float32), (1, 1, 1), eps=0.0)
+    got = torch.from_numpy(out.view(np.int16)).view(torch.bfloat16).double().numpy()[0, 0]
+    want = torch.tensor([1 / math.sqrt(5), 3 / math.sqrt(5)]).to(torch.bfloat16).double().numpy()
+    assert np.array_equal(got[0], np.full(D, want[0])) and np.array_equal(got[1], np.full(D, want[1]))
+
+
+def test_fullnorm_gain_indexes_the_hidden_channel(orc):
+    """gamma has one entry per hidden channel: zero gains on head 1 only silence head 1."""
+    g = torch.Generator().manual_seed(11)
+    x = torch.randn(1, 12, 2, D, generator=g).to(torch.bfloat16)
+    gamma = np.ones(2 * D, np.float32)
+    gamma[D:] = 0.0
+    out = orc.qk_fullnorm_rope_bf16(x, gamma, (1, 3, 4))
+    assert np.all((out[:, :, 1] & 0x7FFF) == 0) and np.any(out[:, :, 0] != 0)
