@@ -268,6 +268,18 @@ def run_gpu(args, rank, world, local):
         if e is not None:
             e[2].record(stream)
     torch.cuda.synchronize()
+    if not wide:
+        # the variant whose RMSNorm spans the whole hidden state, outside the timed step
+        gfq = synth.draw_gamma("gamma_q", rank, heads * 96).to(dev)
+        gfk = synth.draw_gamma("gamma_k", rank, heads * 96).to(dev)
+        fe = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        for i in range(4):
+            if i == 3:
+                fe[0].record(stream)
+            h3a.qk_fullnorm_rope(q, k, gfq, gfk, grid, out=(qn, kn))
+        fe[1].record(stream)
+        torch.cuda.synchronize()
+        kern_ms["prologue_fullnorm"] = allreduce_max(fe[0].elapsed_time(fe[1]), world)
     dit = time_dit_ops(h3a, synth, q, k, B, N, heads * w.head_dim, stream, world, rank)
     if wide:
         kern_ms["prologue"] = kern_ms["prologue_pool"] = 0.0
@@ -373,6 +385,11 @@ def run_gpu(args, rank, world, local):
                                                "traffic": traffic.get("prologue", {}).get("bytes_per_launch")},
             "separate_router_untimed_step": {"ms": round(kern_ms["router"], 4),
                                              "pool_read_GB/s": round(router_gbs, 1)},
+            "prologue_fullwidth_rmsnorm_untimed_step": {
+                "ms": round(kern_ms["prologue_fullnorm"], 4),
+                "GB/s": round(prologue_bytes(N, heads, B) / (kern_ms["prologue_fullnorm"] * 1e-3) / 1e9, 1),
+                "frac_hbm": round(prologue_bytes(N, heads, B) / (kern_ms["prologue_fullnorm"] * 1e-3) / 1e9
+                                  / pk["hbm_gbs"], 4)},
         }) | {
             "attention_sparse": {"ms": round(kern_ms["attention_sparse"], 3), "TFLOP/s": round(sparse_tflops, 2),
                                  "effective_dense_equiv_TFLOP/s":

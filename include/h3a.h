@@ -85,6 +85,19 @@ h3a_status h3a_qk_norm_rope(const void* q, const void* k, const h3a_qkv_desc* d,
  * Returns -1 if sparsity is outside [0, 1) or nkv < 1. */
 int64_t h3a_route_k(int64_t nkv, double sparsity);
 
+/* h3a_qk_norm_rope with the RMSNorm spanning the token's whole hidden state:
+ * the other reading of "QK-RMSNorm" on the same page (fused-operator
+ * paragraph).  For every token n of Q (and of K):
+ *   r = 1 / sqrt(mean over all heads x 96 channels of x^2 + eps)
+ *   y[h, c] = x[h, c] * r * gamma[h * 96 + c], then the per-head 3D RoPE of
+ *   h3a_qk_norm_rope; fp32 arithmetic, one rounding to bf16.
+ * gamma_q/k : fp32 [heads * 96] gains (device, 16-byte aligned).
+ * Other arguments, layouts and errors: as h3a_qk_norm_rope. */
+h3a_status h3a_qk_fullnorm_rope(const void* q, const void* k, const h3a_qkv_desc* d,
+                                const float* gamma_q, const float* gamma_k, h3a_grid grid,
+                                double theta, float eps, void* q_out, void* k_out,
+                                h3a_stream_t stream);
+
 /* Sparsity to use at a denoising step: the router prunes KV blocks from the
  * first_sparse_step-th step on (news.cocoloop.cn MiniMax-H3 SGLang report,
  * SubBlock paragraph: from the 10th step), steps counted from 1.  Returns

@@ -14,10 +14,11 @@ Public API (CUDA tensors, bf16 [B, N, heads, 96]):
 All compute runs in libh3a.so (include/h3a.h); the Python layer only marshals
 arguments.  ``synth`` holds the seeded synthetic input generators.
 """
-from .h3a import (H3AError, attention, attention_core, last_device_error, load, qk_norm_rope, qk_norm_rope_pool,
+from .h3a import (H3AError, attention, attention_core, last_device_error, load, qk_fullnorm_rope, qk_norm_rope,
+                  qk_norm_rope_pool,
                   residual_adaln, residual_diff, route, route_k, route_pooled, route_workspace_size, selftest_exp2,
                   selftest_mma, selftest_wait_timeout, step_sparsity, swiglu)
 
-__all__ = ["H3AError", "attention", "attention_core", "last_device_error", "load", "qk_norm_rope",
+__all__ = ["H3AError", "attention", "attention_core", "last_device_error", "load", "qk_fullnorm_rope", "qk_norm_rope",
            "qk_norm_rope_pool", "residual_adaln", "residual_diff", "route", "route_k", "route_pooled", "route_workspace_size",
            "selftest_exp2", "selftest_mma", "selftest_wait_timeout", "step_sparsity", "swiglu"]

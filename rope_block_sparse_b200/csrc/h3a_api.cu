@@ -183,6 +183,18 @@ double h3a_step_sparsity(int32_t step, int32_t first_sparse_step, double sparsit
     return step >= first_sparse_step ? sparsity : 0.0;
 }
 
+h3a_status h3a_qk_fullnorm_rope(const void* q, const void* k, const h3a_qkv_desc* d, const float* gamma_q,
+                                const float* gamma_k, h3a_grid grid, double theta, float eps, void* q_out,
+                                void* k_out, h3a_stream_t stream) {
+    Shape s;
+    h3a_status rc = prologue_check(q, k, d, gamma_q, gamma_k, grid, theta, eps, q_out, k_out, &s);
+    if (rc != H3A_OK) return rc;
+    if (!aligned16(gamma_q) || !aligned16(gamma_k)) return H3A_ERR_INVALID_ARG;  // read as float4
+    cudaError_t e = launch_qk_fullnorm_rope(q, k, q_out, k_out, gamma_q, gamma_k, s, grid.H, grid.W, theta, eps,
+                                            reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? H3A_OK : cuda_fail(e);
+}
+
 int64_t h3a_route_k(int64_t nkv, double sparsity) {
     if (nkv < 1 || !(sparsity >= 0.0 && sparsity < 1.0)) return -1;
     int64_t kk = static_cast<int64_t>(std::ceil((1.0 - sparsity) * static_cast<double>(nkv) - 1e-9));

@@ -26,6 +26,11 @@ cudaError_t launch_qk_norm_rope(const void* q, const void* k, void* q_out, void*
                                 const float* gamma_k, const Shape& s, int T, int H, int W, double theta,
                                 float eps, cudaStream_t st);
 
+// Prologue whose RMSNorm spans all heads of a token (gains [heads * 96]).
+cudaError_t launch_qk_fullnorm_rope(const void* q, const void* k, void* q_out, void* k_out, const float* gamma_q,
+                                    const float* gamma_k, const Shape& s, int H, int W, double theta, float eps,
+                                    cudaStream_t st);
+
 // Prologue that also writes the fp32 means of its rounded outputs over
 // 128-token blocks into pool_q / pool_k ([B, heads, nblk, 96]) (prologue.cu).
 cudaError_t launch_qk_norm_rope_pool(const void* q, const void* k, void* q_out, void* k_out, const float* gamma_q,

@@ -1,8 +1,9 @@
 // Fused QK-RMSNorm + 3D RoPE prologue (news.cocoloop.cn MiniMax-H3 SGLang
 // report, fused-operator paragraph: QK-RMSNorm with 3D RoPE in one kernel, no
 // change to the result; 3D multimodal RoPE from the 52hbtv.com H3-Image page,
-// section 二, model table), and the same prologue with the router's block
-// pooling folded in (qk_norm_rope_pool_kernel, at the end of this file).
+// section 二, model table), the same prologue with the router's block
+// pooling folded in (qk_norm_rope_pool_kernel), and the variant whose RMSNorm
+// spans the token's whole hidden state (qk_fullnorm_rope_kernel, at the end).
 //
 // HBM-bound: every element of Q and K is read once and written once (4 bytes
 // per element, 43,008 bytes per token at 56 heads).  One warp owns one token at
@@ -291,6 +292,111 @@ __global__ void __launch_bounds__(kPoolThreads, 2) qk_norm_rope_pool_kernel(cons
     }
 }
 
+// ---------------------------------------------------------------------------
+// RMSNorm over the whole hidden state (all heads x 96 channels of a token, one
+// gain per hidden channel), then the same per-head 3D RoPE: the other reading
+// of "QK-RMSNorm" in the fused-operator paragraph.  One warp per token, as in
+// qk_norm_rope_kernel, in two passes: the first sums the squares of all of the
+// token's Q and K channels (a full-warp reduction each), the second reads the
+// row again -- mostly from L2, the row was read an instant earlier -- scales it
+// by the common 1 / RMS and the per-channel gains, rotates and stores.
+__device__ __forceinline__ void scale_rope(const uint2 (&raw)[3], const float (&g)[kChanPerLane], float r,
+                                           const float (&cs)[kPairsPerLane], const float (&sn)[kPairsPerLane],
+                                           uint32_t (&out)[kPairsPerLane]) {
+    float x[kChanPerLane];
+    unpack4(raw[0], x);
+    unpack4(raw[1], x + 4);
+    unpack4(raw[2], x + 8);
+#pragma unroll
+    for (int p = 0; p < kPairsPerLane; ++p) {
+        const float y0 = x[2 * p] * r * g[2 * p];
+        const float y1 = x[2 * p + 1] * r * g[2 * p + 1];
+        const float z0 = y0 * cs[p] - y1 * sn[p];
+        const float z1 = y0 * sn[p] + y1 * cs[p];
+        out[p] = pack2(z0, z1);
+    }
+}
+
+__device__ __forceinline__ float sum_squares(const uint2 (&raw)[3]) {
+    float x[kChanPerLane];
+    unpack4(raw[0], x);
+    unpack4(raw[1], x + 4);
+    unpack4(raw[2], x + 8);
+    float ss = 0.f;
+#pragma unroll
+    for (int i = 0; i < kChanPerLane; ++i) ss = fmaf(x[i], x[i], ss);
+    return ss;
+}
+
+__device__ __forceinline__ void load_gain(const float* g, float (&o)[kChanPerLane]) {
+    const float4* v = reinterpret_cast<const float4*>(g);
+#pragma unroll
+    for (int u = 0; u < 3; ++u) {
+        const float4 t = __ldg(v + u);
+        o[4 * u] = t.x, o[4 * u + 1] = t.y, o[4 * u + 2] = t.z, o[4 * u + 3] = t.w;
+    }
+}
+
+__global__ void __launch_bounds__(kThreads, 3) qk_fullnorm_rope_kernel(const PrologueArgs a) {
+    const int lane = threadIdx.x & 31;
+    const int grp = lane >> 3;
+    const int sub = lane & 7;
+    const int c0 = sub * kChanPerLane;
+    const int64_t warps = static_cast<int64_t>(gridDim.x) * (kThreads / 32);
+    const int head_groups = (a.heads + 3) >> 2;
+    const float inv_width = 1.0f / static_cast<float>(a.heads * kHeadDim);
+    for (int64_t tok = static_cast<int64_t>(blockIdx.x) * (kThreads / 32) + (threadIdx.x >> 5); tok < a.tokens;
+         tok += warps) {
+        const int b = static_cast<int>(tok / a.N);
+        const int n = static_cast<int>(tok - static_cast<int64_t>(b) * a.N);
+        const int64_t tok_off = static_cast<int64_t>(b) * a.sb + static_cast<int64_t>(n) * a.sn + c0;
+        // pass 1: sums of squares over the whole hidden state of Q and of K
+        float ssq = 0.f, ssk = 0.f;
+        for (int hg = 0; hg < head_groups; ++hg) {
+            const int h = hg * 4 + grp;
+            const bool act = h < a.heads;
+            const int64_t off = tok_off + static_cast<int64_t>(h) * a.sh;
+            uint2 rq[3], rk[3];
+            load3(a.q + off, act, rq);
+            load3(a.k + off, act, rk);
+            ssq += sum_squares(rq);
+            ssk += sum_squares(rk);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            ssq += __shfl_xor_sync(0xffffffffu, ssq, o);
+            ssk += __shfl_xor_sync(0xffffffffu, ssk, o);
+        }
+        const float rq_ = rsqrtf(ssq * inv_width + a.eps);
+        const float rk_ = rsqrtf(ssk * inv_width + a.eps);
+
+        const int pt = n / (a.H * a.W), ph = (n / a.W) % a.H, pw = n % a.W;
+        float cs[kPairsPerLane], sn[kPairsPerLane];
+#pragma unroll
+        for (int p = 0; p < kPairsPerLane; ++p)
+            rotation(pt, ph, pw, sub * kPairsPerLane + p, a.freq_hi, a.freq_lo, cs[p], sn[p]);
+        // pass 2: scale, rotate, store
+        for (int hg = 0; hg < head_groups; ++hg) {
+            const int h = hg * 4 + grp;
+            const bool act = h < a.heads;
+            const int64_t off = tok_off + static_cast<int64_t>(h) * a.sh;
+            uint2 rq[3], rk[3];
+            load3(a.q + off, act, rq);
+            load3(a.k + off, act, rk);
+            if (act) {
+                float gq[kChanPerLane], gk[kChanPerLane];
+                load_gain(a.gq + h * kHeadDim + c0, gq);
+                load_gain(a.gk + h * kHeadDim + c0, gk);
+                uint32_t oq[kPairsPerLane], ok[kPairsPerLane];
+                scale_rope(rq, gq, rq_, cs, sn, oq);
+                scale_rope(rk, gk, rk_, cs, sn, ok);
+                store3(oq, true, a.qo + off);
+                store3(ok, true, a.ko + off);
+            }
+        }
+    }
+}
+
 }  // namespace
 
 namespace {
@@ -369,6 +475,39 @@ cudaError_t launch_qk_norm_rope_pool(const void* q, const void* k, void* q_out, 
                                          static_cast<int>(kPoolSmemBytes));
     if (e != cudaSuccess) return e;
     qk_norm_rope_pool_kernel<<<dim3(a.nblk, s.B, chunks), kPoolThreads, kPoolSmemBytes, st>>>(a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_qk_fullnorm_rope(const void* q, const void* k, void* q_out, void* k_out, const float* gamma_q,
+                                    const float* gamma_k, const Shape& s, int H, int W, double theta, float eps,
+                                    cudaStream_t st) {
+    PrologueArgs a;
+    a.q = static_cast<const __nv_bfloat16*>(q);
+    a.k = static_cast<const __nv_bfloat16*>(k);
+    a.qo = static_cast<__nv_bfloat16*>(q_out);
+    a.ko = static_cast<__nv_bfloat16*>(k_out);
+    a.gq = gamma_q;
+    a.gk = gamma_k;
+    a.tokens = static_cast<int64_t>(s.B) * s.N;
+    a.N = s.N;
+    a.heads = s.heads;
+    a.H = H;
+    a.W = W;
+    a.sb = s.sb;
+    a.sn = s.sn;
+    a.sh = s.sh;
+    a.eps = eps;
+    set_frequencies(theta, a);
+    a.pool_q = a.pool_k = nullptr;
+    a.nblk = 0;
+    if (a.tokens == 0) return cudaSuccess;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    int64_t blocks = (a.tokens + (kThreads / 32) - 1) / (kThreads / 32);
+    const int64_t cap = static_cast<int64_t>(sms) * 3 * 8;
+    if (blocks > cap) blocks = cap;
+    qk_fullnorm_rope_kernel<<<static_cast<unsigned>(blocks), kThreads, 0, st>>>(a);
     return cudaGetLastError();
 }
 

@@ -27,7 +27,7 @@ EXPORTS = ("h3a_qk_norm_rope", "h3a_route_k", "h3a_route_workspace_size", "h3a_r
            "h3a_status_string", "h3a_last_cuda_error_string", "h3a_last_device_error",
            "h3a_selftest_wait_timeout", "h3a_selftest_mma", "h3a_selftest_exp2", "h3a_route_noalloc",
            "h3a_qk_norm_rope_pool", "h3a_route_pooled", "h3a_residual_adaln", "h3a_swiglu",
-           "h3a_residual_diff", "h3a_step_sparsity")
+           "h3a_residual_diff", "h3a_step_sparsity", "h3a_qk_fullnorm_rope")
 ROUTE_NOALLOC_MAX_BYTES = 64 << 20  # H3A_ROUTE_NOALLOC_MAX_BYTES
 RESIDUAL_DIFF_WORKSPACE_BYTES = 32768  # H3A_RESIDUAL_DIFF_WORKSPACE_BYTES
 
@@ -104,6 +104,8 @@ def load() -> ctypes.CDLL:
     lib.h3a_residual_diff.restype = st
     lib.h3a_step_sparsity.argtypes = [i32, i32, f64]
     lib.h3a_step_sparsity.restype = f64
+    lib.h3a_qk_fullnorm_rope.argtypes = [P, P, ctypes.POINTER(QkvDesc), P, P, Grid, f64, f32, P, P, P]
+    lib.h3a_qk_fullnorm_rope.restype = st
     _lib = lib
     return lib
 
@@ -168,6 +170,30 @@ def qk_norm_rope(q: torch.Tensor, k: torch.Tensor, gamma_q: torch.Tensor, gamma_
     _check("h3a_qk_norm_rope", lib.h3a_qk_norm_rope(_ptr(q), _ptr(k), ctypes.byref(d), _ptr(gamma_q),
                                                     _ptr(gamma_k), Grid(*grid), float(theta), float(eps),
                                                     _ptr(qo), _ptr(ko), _stream_handle()))
+    return qo, ko
+
+
+def qk_fullnorm_rope(q: torch.Tensor, k: torch.Tensor, gamma_q: torch.Tensor, gamma_k: torch.Tensor, grid,
+                     theta: float = 10000.0, eps: float = 1e-6, inplace: bool = False, out=None):
+    """qk_norm_rope with the RMSNorm over each token's whole hidden state (all heads);
+    gamma_q, gamma_k: fp32 [heads * 96].  Returns (q_out, k_out)."""
+    lib = load()
+    _check_qkv(q, k)
+    heads = q.shape[2]
+    for g in (gamma_q, gamma_k):
+        if not g.is_cuda or g.dtype != torch.float32 or g.numel() != heads * HEAD_DIM or not g.is_contiguous():
+            raise ValueError("gammas must be contiguous fp32 [heads * 96] CUDA tensors")
+    if inplace:
+        qo, ko = q, k
+    elif out is not None:
+        qo, ko = out
+        _check_qkv(q, qo, ko)
+    else:
+        qo, ko = torch.empty_like(q), torch.empty_like(k)
+    d = desc_of(q)
+    _check("h3a_qk_fullnorm_rope", lib.h3a_qk_fullnorm_rope(_ptr(q), _ptr(k), ctypes.byref(d), _ptr(gamma_q),
+                                                            _ptr(gamma_k), Grid(*grid), float(theta), float(eps),
+                                                            _ptr(qo), _ptr(ko), _stream_handle()))
     return qo, ko
 
 
