@@ -59,26 +59,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
-// try_wait with an explicit suspend-time hint: the thread sleeps until the
-// phase completes or about `hint_ns` has passed, instead of the
-// implementation-defined default.
-__device__ __forceinline__ bool mbar_try_wait_hint(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
-        : "memory");
-    return ok != 0;
-}
-
-// Suspend-time hint of the polling loop (ns); 0 keeps the default.
-#ifndef H3A_WAIT_HINT_NS
-#define H3A_WAIT_HINT_NS 0
-#endif
-
 // Bounded wait: true once the phase of parity `parity` completed; false when
 // the CTA-wide abort flag is raised or `limit_ns` elapses (the caller then
 // raises the abort flag and leaves its loop).  Fully inlined: an out-of-line
@@ -90,8 +70,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     for (uint32_t i = 1;; ++i) {
-        if (H3A_WAIT_HINT_NS > 0 ? mbar_try_wait_hint(bar, parity, H3A_WAIT_HINT_NS) : mbar_try_wait(bar, parity))
-            return true;
+        if (mbar_try_wait(bar, parity)) return true;
         if ((i & 15u) == 0u) {
             if (*abort_flag) return false;
             if (global_timer_ns() - t0 > limit_ns) return false;
