@@ -92,7 +92,9 @@ int64_t h3a_route_k(int64_t nkv, double sparsity);
  *   y[h, c] = x[h, c] * r * gamma[h * 96 + c], then the per-head 3D RoPE of
  *   h3a_qk_norm_rope; fp32 arithmetic, one rounding to bf16.
  * gamma_q/k : fp32 [heads * 96] gains (device, 16-byte aligned).
- * Other arguments, layouts and errors: as h3a_qk_norm_rope. */
+ * Other arguments, layouts and errors: as h3a_qk_norm_rope, and UNSUPPORTED
+ * for more than 74 heads or B * N >= 2^31 (one CTA per token holds the
+ * token's rows). */
 h3a_status h3a_qk_fullnorm_rope(const void* q, const void* k, const h3a_qkv_desc* d,
                                 const float* gamma_q, const float* gamma_k, h3a_grid grid,
                                 double theta, float eps, void* q_out, void* k_out,

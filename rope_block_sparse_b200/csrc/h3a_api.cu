@@ -190,6 +190,8 @@ h3a_status h3a_qk_fullnorm_rope(const void* q, const void* k, const h3a_qkv_desc
     h3a_status rc = prologue_check(q, k, d, gamma_q, gamma_k, grid, theta, eps, q_out, k_out, &s);
     if (rc != H3A_OK) return rc;
     if (!aligned16(gamma_q) || !aligned16(gamma_k)) return H3A_ERR_INVALID_ARG;  // read as float4
+    // one CTA per token, each holding its token's rows in registers
+    if (s.heads > 74 || static_cast<int64_t>(s.B) * s.N >= (int64_t(1) << 31)) return H3A_ERR_UNSUPPORTED;
     cudaError_t e = launch_qk_fullnorm_rope(q, k, q_out, k_out, gamma_q, gamma_k, s, grid.H, grid.W, theta, eps,
                                             reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? H3A_OK : cuda_fail(e);

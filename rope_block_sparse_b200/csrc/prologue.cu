@@ -295,105 +295,99 @@ __global__ void __launch_bounds__(kPoolThreads, 2) qk_norm_rope_pool_kernel(cons
 // ---------------------------------------------------------------------------
 // RMSNorm over the whole hidden state (all heads x 96 channels of a token, one
 // gain per hidden channel), then the same per-head 3D RoPE: the other reading
-// of "QK-RMSNorm" in the fused-operator paragraph.  One warp per token, as in
-// qk_norm_rope_kernel, in two passes: the first sums the squares of all of the
-// token's Q and K channels (a full-warp reduction each), the second reads the
-// row again -- mostly from L2, the row was read an instant earlier -- scales it
-// by the common 1 / RMS and the per-channel gains, rotates and stores.
-__device__ __forceinline__ void scale_rope(const uint2 (&raw)[3], const float (&g)[kChanPerLane], float r,
-                                           const float (&cs)[kPairsPerLane], const float (&sn)[kPairsPerLane],
-                                           uint32_t (&out)[kPairsPerLane]) {
-    float x[kChanPerLane];
-    unpack4(raw[0], x);
-    unpack4(raw[1], x + 4);
-    unpack4(raw[2], x + 8);
-#pragma unroll
-    for (int p = 0; p < kPairsPerLane; ++p) {
-        const float y0 = x[2 * p] * r * g[2 * p];
-        const float y1 = x[2 * p + 1] * r * g[2 * p + 1];
-        const float z0 = y0 * cs[p] - y1 * sn[p];
-        const float z1 = y0 * sn[p] + y1 * cs[p];
-        out[p] = pack2(z0, z1);
+// of "QK-RMSNorm" in the fused-operator paragraph.  One 224-thread CTA per
+// token keeps the token's Q and K rows in registers (16-byte vector v of a row
+// = head v / 12, channels 8 * (v % 12) .. + 7; three vectors per thread per
+// tensor at 56 heads), so each row is read from HBM once: sums of squares of
+// Q and of K reduced over the CTA, the token's 48 rotations computed once into
+// shared memory, then scale, rotate and store.
+constexpr int kFullThreads = 224;
+constexpr int kFullWarps = kFullThreads / 32;
+constexpr int kVecPerHead = kHeadDim / 8;  // 12
+
+template <int VPT>
+__global__ void __launch_bounds__(kFullThreads) qk_fullnorm_rope_kernel(const PrologueArgs a) {
+    __shared__ float2 rot[kPairsPerHead];
+    __shared__ float red[2][kFullWarps];
+    const int64_t tok = blockIdx.x;
+    const int b = static_cast<int>(tok / a.N);
+    const int n = static_cast<int>(tok - static_cast<int64_t>(b) * a.N);
+    if (threadIdx.x < kPairsPerHead) {
+        float c, sn;
+        rotation(n / (a.H * a.W), (n / a.W) % a.H, n % a.W, threadIdx.x, a.freq_hi, a.freq_lo, c, sn);
+        rot[threadIdx.x] = make_float2(c, sn);
     }
-}
-
-__device__ __forceinline__ float sum_squares(const uint2 (&raw)[3]) {
-    float x[kChanPerLane];
-    unpack4(raw[0], x);
-    unpack4(raw[1], x + 4);
-    unpack4(raw[2], x + 8);
-    float ss = 0.f;
+    const int nvec = a.heads * kVecPerHead;
+    const int64_t tok_off = static_cast<int64_t>(b) * a.sb + static_cast<int64_t>(n) * a.sn;
+    uint4 xq[VPT], xk[VPT];
+    float ssq = 0.f, ssk = 0.f;
 #pragma unroll
-    for (int i = 0; i < kChanPerLane; ++i) ss = fmaf(x[i], x[i], ss);
-    return ss;
-}
-
-__device__ __forceinline__ void load_gain(const float* g, float (&o)[kChanPerLane]) {
-    const float4* v = reinterpret_cast<const float4*>(g);
+    for (int u = 0; u < VPT; ++u) {
+        const int v = threadIdx.x + u * kFullThreads;
+        xq[u] = xk[u] = make_uint4(0, 0, 0, 0);
+        if (v < nvec) {
+            const int64_t off = tok_off + static_cast<int64_t>(v / kVecPerHead) * a.sh + (v % kVecPerHead) * 8;
+            xq[u] = __ldg(reinterpret_cast<const uint4*>(a.q + off));
+            xk[u] = __ldg(reinterpret_cast<const uint4*>(a.k + off));
+        }
+        const uint32_t wq[4] = {xq[u].x, xq[u].y, xq[u].z, xq[u].w};
+        const uint32_t wk[4] = {xk[u].x, xk[u].y, xk[u].z, xk[u].w};
 #pragma unroll
-    for (int u = 0; u < 3; ++u) {
-        const float4 t = __ldg(v + u);
-        o[4 * u] = t.x, o[4 * u + 1] = t.y, o[4 * u + 2] = t.z, o[4 * u + 3] = t.w;
+        for (int i = 0; i < 4; ++i) {
+            const float q0 = __uint_as_float(wq[i] << 16), q1 = __uint_as_float(wq[i] & 0xFFFF0000u);
+            const float k0 = __uint_as_float(wk[i] << 16), k1 = __uint_as_float(wk[i] & 0xFFFF0000u);
+            ssq = fmaf(q0, q0, fmaf(q1, q1, ssq));
+            ssk = fmaf(k0, k0, fmaf(k1, k1, ssk));
+        }
     }
-}
-
-__global__ void __launch_bounds__(kThreads, 3) qk_fullnorm_rope_kernel(const PrologueArgs a) {
-    const int lane = threadIdx.x & 31;
-    const int grp = lane >> 3;
-    const int sub = lane & 7;
-    const int c0 = sub * kChanPerLane;
-    const int64_t warps = static_cast<int64_t>(gridDim.x) * (kThreads / 32);
-    const int head_groups = (a.heads + 3) >> 2;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        ssq += __shfl_xor_sync(0xffffffffu, ssq, o);
+        ssk += __shfl_xor_sync(0xffffffffu, ssk, o);
+    }
+    if ((threadIdx.x & 31) == 0) {
+        red[0][threadIdx.x >> 5] = ssq;
+        red[1][threadIdx.x >> 5] = ssk;
+    }
+    __syncthreads();  // also publishes rot[]
+    ssq = ssk = 0.f;
+#pragma unroll
+    for (int w = 0; w < kFullWarps; ++w) {
+        ssq += red[0][w];
+        ssk += red[1][w];
+    }
     const float inv_width = 1.0f / static_cast<float>(a.heads * kHeadDim);
-    for (int64_t tok = static_cast<int64_t>(blockIdx.x) * (kThreads / 32) + (threadIdx.x >> 5); tok < a.tokens;
-         tok += warps) {
-        const int b = static_cast<int>(tok / a.N);
-        const int n = static_cast<int>(tok - static_cast<int64_t>(b) * a.N);
-        const int64_t tok_off = static_cast<int64_t>(b) * a.sb + static_cast<int64_t>(n) * a.sn + c0;
-        // pass 1: sums of squares over the whole hidden state of Q and of K
-        float ssq = 0.f, ssk = 0.f;
-        for (int hg = 0; hg < head_groups; ++hg) {
-            const int h = hg * 4 + grp;
-            const bool act = h < a.heads;
-            const int64_t off = tok_off + static_cast<int64_t>(h) * a.sh;
-            uint2 rq[3], rk[3];
-            load3(a.q + off, act, rq);
-            load3(a.k + off, act, rk);
-            ssq += sum_squares(rq);
-            ssk += sum_squares(rk);
-        }
+    const float rq = rsqrtf(ssq * inv_width + a.eps);
+    const float rk = rsqrtf(ssk * inv_width + a.eps);
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            ssq += __shfl_xor_sync(0xffffffffu, ssq, o);
-            ssk += __shfl_xor_sync(0xffffffffu, ssk, o);
-        }
-        const float rq_ = rsqrtf(ssq * inv_width + a.eps);
-        const float rk_ = rsqrtf(ssk * inv_width + a.eps);
-
-        const int pt = n / (a.H * a.W), ph = (n / a.W) % a.H, pw = n % a.W;
-        float cs[kPairsPerLane], sn[kPairsPerLane];
+    for (int u = 0; u < VPT; ++u) {
+        const int v = threadIdx.x + u * kFullThreads;
+        if (v >= nvec) continue;
+        const int h = v / kVecPerHead, c0 = (v % kVecPerHead) * 8;
+        const int64_t off = tok_off + static_cast<int64_t>(h) * a.sh + c0;
+        float gq[8], gk[8];
+        const float4* pq = reinterpret_cast<const float4*>(a.gq + h * kHeadDim + c0);
+        const float4* pk = reinterpret_cast<const float4*>(a.gk + h * kHeadDim + c0);
+        const float4 gq0 = __ldg(pq), gq1 = __ldg(pq + 1), gk0 = __ldg(pk), gk1 = __ldg(pk + 1);
+        gq[0] = gq0.x, gq[1] = gq0.y, gq[2] = gq0.z, gq[3] = gq0.w, gq[4] = gq1.x, gq[5] = gq1.y, gq[6] = gq1.z,
+        gq[7] = gq1.w;
+        gk[0] = gk0.x, gk[1] = gk0.y, gk[2] = gk0.z, gk[3] = gk0.w, gk[4] = gk1.x, gk[5] = gk1.y, gk[6] = gk1.z,
+        gk[7] = gk1.w;
+        const uint32_t wq[4] = {xq[u].x, xq[u].y, xq[u].z, xq[u].w};
+        const uint32_t wk[4] = {xk[u].x, xk[u].y, xk[u].z, xk[u].w};
+        uint32_t oq[4], ok[4];
 #pragma unroll
-        for (int p = 0; p < kPairsPerLane; ++p)
-            rotation(pt, ph, pw, sub * kPairsPerLane + p, a.freq_hi, a.freq_lo, cs[p], sn[p]);
-        // pass 2: scale, rotate, store
-        for (int hg = 0; hg < head_groups; ++hg) {
-            const int h = hg * 4 + grp;
-            const bool act = h < a.heads;
-            const int64_t off = tok_off + static_cast<int64_t>(h) * a.sh;
-            uint2 rq[3], rk[3];
-            load3(a.q + off, act, rq);
-            load3(a.k + off, act, rk);
-            if (act) {
-                float gq[kChanPerLane], gk[kChanPerLane];
-                load_gain(a.gq + h * kHeadDim + c0, gq);
-                load_gain(a.gk + h * kHeadDim + c0, gk);
-                uint32_t oq[kPairsPerLane], ok[kPairsPerLane];
-                scale_rope(rq, gq, rq_, cs, sn, oq);
-                scale_rope(rk, gk, rk_, cs, sn, ok);
-                store3(oq, true, a.qo + off);
-                store3(ok, true, a.ko + off);
-            }
+        for (int i = 0; i < 4; ++i) {
+            const float2 cs = rot[c0 / 2 + i];  // pair (c0 + 2i, c0 + 2i + 1) of the head
+            const float q0 = __uint_as_float(wq[i] << 16) * rq * gq[2 * i];
+            const float q1 = __uint_as_float(wq[i] & 0xFFFF0000u) * rq * gq[2 * i + 1];
+            const float k0 = __uint_as_float(wk[i] << 16) * rk * gk[2 * i];
+            const float k1 = __uint_as_float(wk[i] & 0xFFFF0000u) * rk * gk[2 * i + 1];
+            oq[i] = pack2(q0 * cs.x - q1 * cs.y, q0 * cs.y + q1 * cs.x);
+            ok[i] = pack2(k0 * cs.x - k1 * cs.y, k0 * cs.y + k1 * cs.x);
         }
+        *reinterpret_cast<uint4*>(a.qo + off) = make_uint4(oq[0], oq[1], oq[2], oq[3]);
+        *reinterpret_cast<uint4*>(a.ko + off) = make_uint4(ok[0], ok[1], ok[2], ok[3]);
     }
 }
 
@@ -501,13 +495,14 @@ cudaError_t launch_qk_fullnorm_rope(const void* q, const void* k, void* q_out, v
     a.pool_q = a.pool_k = nullptr;
     a.nblk = 0;
     if (a.tokens == 0) return cudaSuccess;
-    int dev = 0, sms = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    int64_t blocks = (a.tokens + (kThreads / 32) - 1) / (kThreads / 32);
-    const int64_t cap = static_cast<int64_t>(sms) * 3 * 8;
-    if (blocks > cap) blocks = cap;
-    qk_fullnorm_rope_kernel<<<static_cast<unsigned>(blocks), kThreads, 0, st>>>(a);
+    const unsigned grid = static_cast<unsigned>(a.tokens);
+    switch ((s.heads * kVecPerHead + kFullThreads - 1) / kFullThreads) {
+        case 1: qk_fullnorm_rope_kernel<1><<<grid, kFullThreads, 0, st>>>(a); break;
+        case 2: qk_fullnorm_rope_kernel<2><<<grid, kFullThreads, 0, st>>>(a); break;
+        case 3: qk_fullnorm_rope_kernel<3><<<grid, kFullThreads, 0, st>>>(a); break;
+        case 4: qk_fullnorm_rope_kernel<4><<<grid, kFullThreads, 0, st>>>(a); break;
+        default: return cudaErrorNotSupported;  // more than 74 heads
+    }
     return cudaGetLastError();
 }
 
