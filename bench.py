@@ -429,6 +429,7 @@ def run_gpu(args, rank, world, local):
             "separate_router_untimed_step": {"ms": round(kern_ms["router"], 4),
                                              "pool_read_GB/s": round(router_gbs, 1)},
             "prologue_fullwidth_rmsnorm_untimed_step": {
+                "traffic": traffic.get("prologue_fullnorm", {}).get("bytes_per_launch"),
                 "ms": round(kern_ms["prologue_fullnorm"], 4),
                 "GB/s": round(prologue_bytes(N, heads, B) / (kern_ms["prologue_fullnorm"] * 1e-3) / 1e9, 1),
                 "frac_hbm": round(prologue_bytes(N, heads, B) / (kern_ms["prologue_fullnorm"] * 1e-3) / 1e9
@@ -441,7 +442,9 @@ def run_gpu(args, rank, world, local):
             "attention_dense": {"ms": round(kern_ms["attention_dense"], 3), "TFLOP/s": round(dense_tflops, 2)},
             "sparse_speedup_incl_router": round(kern_ms["attention_dense"] /
                                                 (kern_ms["attention_sparse"] + route_cost), 3),
-        } | {name: dict(ent, frac_hbm=round(ent["GB/s"] / pk["hbm_gbs"], 4)) for name, ent in dit.items()},
+        } | {name: dict(ent, frac_hbm=round(ent["GB/s"] / pk["hbm_gbs"], 4),
+                        traffic=traffic.get(ent.pop("traffic_key"), {}).get("bytes_per_launch"))
+             for name, ent in dit.items()},
         "gpu_launches": args.steps * 4,
         "clocks": clocks,
         "e2e": e2e,
@@ -491,11 +494,14 @@ def time_dit_ops(h3a, synth, q, k, B, N, width, stream, world, rank, reps=10):
     rows = B * N
     return {
         "dit_residual_adaln_untimed_step": {"ms": round(ms_ad, 4), "rows": rows, "width": width,
-                                            "GB/s": round(8.0 * rows * width / (ms_ad * 1e-3) / 1e9, 1)},
+                                            "GB/s": round(8.0 * rows * width / (ms_ad * 1e-3) / 1e9, 1),
+                                            "traffic_key": "residual_adaln"},
         "dit_swiglu_untimed_step": {"ms": round(ms_sw, 4), "rows": rows, "ffn_width": ffn,
-                                    "GB/s": round(6.0 * rows * ffn / (ms_sw * 1e-3) / 1e9, 1)},
+                                    "GB/s": round(6.0 * rows * ffn / (ms_sw * 1e-3) / 1e9, 1),
+                                    "traffic_key": "swiglu"},
         "cache_dit_residual_diff_untimed_step": {"ms": round(ms_rd, 4), "values": rows * width,
-                                                 "GB/s": round(4.0 * rows * width / (ms_rd * 1e-3) / 1e9, 1)},
+                                                 "GB/s": round(4.0 * rows * width / (ms_rd * 1e-3) / 1e9, 1),
+                                                 "traffic_key": "residual_diff"},
     }
 
 
