@@ -61,3 +61,12 @@ def test_flop_counts():
     all_blocks = np.broadcast_to(np.arange(nblk, dtype=np.int32), (1, 2, nblk, nblk))
     assert bench.attention_flops(N, 2, 1, blocks=all_blocks) == pytest.approx(bench.attention_flops(N, 2, 1))
     assert bench.prologue_bytes(124992, 56, 1) == 124992 * 43008
+
+
+def test_wide_workload_counts():
+    """42 heads x 128 carry the same hidden width as 56 x 96, hence the same dense
+    FLOPs; the fused prologue's pooled means are 2 x 4 B per (head, block, channel)."""
+    w = synth.WORKLOADS["video5s_d128"]
+    assert w.heads * w.head_dim == 56 * 96
+    assert bench.attention_flops(w.N, w.heads, w.B, d=w.head_dim) == bench.attention_flops(w.N, 56, 1)
+    assert bench.pooled_bytes(124992, 56, 1) == 2 * 4 * 56 * 977 * 96
