@@ -9,22 +9,22 @@
 // 2p and 2p+1, i.e. the router's query blocks -- and streams 128-row K/V tiles
 // through shared memory: every KV block for dense attention, or each tile's
 // own routed list in sparse mode (a KV tile both lists name at the same step is
-// loaded once and shared).  Warp roles (576 threads, 18 warps):
-//   warps 0-15  softmax: warpgroup g = warp / 4 handles query tile g / 2 and key
-//               columns [64 (g % 2), 64 (g % 2) + 64) of every 128-key block;
-//               thread r owns row r (TMEM lane r) of that half.  It reads its 64
-//               S values from TMEM, computes exp2 in fp32 (log2 domain) with the
-//               row's reference max, writes P as packed bf16 over the first 32
-//               columns of its own S half, and agrees with the other half on the
-//               row max through shared memory and a bounded mbarrier.  The
-//               reference is fixed by the first block; a later block recomputes
-//               its P and rescales O only when a row max grew by more than 2^8
-//               (the final division by the row sum keeps this exact).  At the end
-//               each half divides its 48 O columns by the row sum, rounds once to
-//               bf16 and stores them.
-//   warp 16     TMA producer: Q tiles once, then a 3-stage K ring and a 3-stage
+// loaded once and shared).  Warp roles (320 threads, 10 warps):
+//   warps 0-7   softmax: warpgroup t = warp / 4 handles query tile t; thread r
+//               owns row r (TMEM lane r) and all 128 key columns of every
+//               block, so the row max and row sum never leave the thread.  It
+//               loads the whole row of S from TMEM with one wait, takes the
+//               block max, computes exp2 in fp32 (log2 domain, packed f32x2
+//               FMAs and adds) against the row's reference max, packs P to bf16
+//               in place over the same registers and writes it over the first
+//               64 columns of S.  The reference is fixed by the first block; a
+//               later block moves it up and rescales O (in TMEM) only when the
+//               row max grew by more than 2^8 (the final division by the row
+//               sum keeps this exact).  At the end the thread divides its O row
+//               by the row sum, rounds once to bf16 and stores it.
+//   warp 8      TMA producer: Q tiles once, then a 3-stage K ring and a 3-stage
 //               V ring (64-byte swizzled 128 x 32 chunks, 3 per 128 x 96 tile).
-//   warp 17     owns tensor memory (512 columns) and issues tcgen05.mma from one
+//   warp 9      owns tensor memory (512 columns) and issues tcgen05.mma from one
 //               thread: S_t = Q_t K^T (M=128, N=128, K=96 as 6 steps of 16) into
 //               TMEM, O_t += P_t V (M=128, N=96, K=128 as 8 steps, P read from
 //               TMEM, V as an MN-major operand).  Order per step j:
@@ -38,14 +38,15 @@
 #include <cuda_bf16.h>
 
 #include "h3a_internal.h"
+#include "fastmath.cuh"
 #include "sm100.cuh"
 
 namespace h3a {
 namespace {
 
-constexpr int kSoftmaxWarps = 16;                  // 4 warpgroups: (tile, column half)
-constexpr int kProducerWarp = 16, kMmaWarp = 17;
-constexpr int kThreads = 32 * (kSoftmaxWarps + 2);  // 576
+constexpr int kSoftmaxWarps = 8;                   // 2 warpgroups: one per query tile
+constexpr int kProducerWarp = 8, kMmaWarp = 9;
+constexpr int kThreads = 32 * (kSoftmaxWarps + 2);  // 320
 constexpr int kChunkBytes = 128 * 64;        // 128 rows x 32 bf16, 64-byte swizzle
 constexpr uint32_t kTmemCols = 512;
 // TMEM column of S_t
@@ -63,7 +64,6 @@ struct Geo {
     static constexpr int kTileBytes = kChunks * kChunkBytes;
     static constexpr int kStages = D == 96 ? 3 : 2;
     static constexpr int kKSteps = D / 16;  // QK^T k-steps of 16
-    static constexpr int kHalf = D / 2;     // O columns per softmax half
     __host__ __device__ static constexpr uint32_t col_o(int t) { return 256u + (t ? D : 0); }
 };
 
@@ -78,23 +78,11 @@ struct AttnSmem {
     uint64_t k_full[kStages], k_empty[kStages];
     uint64_t v_full[kStages], v_empty[kStages];
     uint64_t s_full[2], p_full[2], o_done[2];
-    uint64_t xbar[2][2];         // [buffer][tile]: half-row maxima exchanged
-    uint64_t lbar[2];            // [tile]: half-row sums exchanged at the end
     uint64_t mma_drain;
-    float xmax[2][2][2][128];    // [buffer][tile][half][row]
-    float lsum[2][2][128];       // [tile][half][row]
     uint32_t tmem_base;
     int abort_flag;
     int never;  // stays 0: abort flag for waits that must ignore an abort
 };
-
-// tcgen05.ld / st of 16 or 32 columns, chosen by the register array's size.
-__device__ __forceinline__ void tmem_ld_n(uint32_t a, uint32_t (&r)[16]) { tmem_ld_x16(a, r); }
-__device__ __forceinline__ void tmem_ld_n(uint32_t a, uint32_t (&r)[32]) { tmem_ld_x32(a, r); }
-__device__ __forceinline__ void tmem_wait_ld_n(uint32_t (&r)[16]) { tmem_wait_ld_x16(r); }
-__device__ __forceinline__ void tmem_wait_ld_n(uint32_t (&r)[32]) { tmem_wait_ld_x32(r); }
-__device__ __forceinline__ void tmem_st_n(uint32_t a, const uint32_t (&r)[16]) { tmem_st_x16(a, r); }
-__device__ __forceinline__ void tmem_st_n(uint32_t a, const uint32_t (&r)[32]) { tmem_st_x32(a, r); }
 
 template <int D>
 constexpr size_t smem_bytes() { return sizeof(AttnSmem<D>) + 1024; }  // + alignment slack
@@ -268,10 +256,10 @@ __device__ __forceinline__ bool issue_pv(AttnSmem<D>& sm, const AttnArgs& a, Mma
     constexpr uint32_t idesc = idesc_bf16_f32(128, D, 0, 1);
     const uint64_t dv = st.dv + stage * stage_step<D>();
     const uint32_t d = tmem + Geo<D>::col_o(t), pa = tmem + col_s(t);
-    // keys 0..63: P at S columns [0, 32); keys 64..127: P at S columns [64, 96)
+    // P_t: keys 2c and 2c+1 packed in S column c
     mma_ts(d, pa, dv, idesc, first ? 0u : 1u);
 #pragma unroll
-    for (int s = 1; s < 8; ++s) mma_ts(d, pa + 64 * (s >> 2) + 8 * (s & 3), dv + mnmajor_step(s), idesc, 1u);
+    for (int s = 1; s < 8; ++s) mma_ts(d, pa + 8 * s, dv + mnmajor_step(s), idesc, 1u);
     if (t == 1 || !p.shared) tc_commit(&sm.v_empty[stage]);
     return true;
 }
@@ -321,48 +309,37 @@ __device__ void mma_issuer(AttnSmem<D>& sm, const AttnArgs& a, uint32_t tmem, bo
     mbar_wait(&sm.mma_drain, 0u, never, a.timeout_ns);
 }
 
-// Exponentials of one 64-key half row with reference m: P packed to bf16 into
-// the first 32 columns of this half's S region; returns the partial sums.
-__device__ __forceinline__ float exp_store_half(const uint32_t (&s)[2][32], float c, float m, uint32_t tS,
-                                                float* hmax) {
-    const float neg_m = -m;
-    float pm[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-    float ps[4] = {0.f, 0.f, 0.f, 0.f};
+// tcgen05.ld of 32 columns into / wait on a 32-register slice of a longer row.
+__device__ __forceinline__ uint32_t (&slice32(uint32_t* x))[32] { return *reinterpret_cast<uint32_t(*)[32]>(x); }
+
+// O row *= alpha (rare rescale).  Out of line: it runs only when a row max
+// grows by more than 2^8, and its registers stay out of the steady-state loop.
+template <int D>
+__device__ __noinline__ void rescale_o(uint32_t tO, float alpha) {
+#pragma unroll 1
+    for (int cc = 0; cc < Geo<D>::kChunks; ++cc) {
+        uint32_t o[32];
+        tmem_ld_x32(tO + 32u * cc, o);
+        tmem_wait_ld_x32(o);
 #pragma unroll
-    for (int q2 = 0; q2 < 2; ++q2) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const float x0 = __uint_as_float(s[q2][2 * i]), x1 = __uint_as_float(s[q2][2 * i + 1]);
-            if (hmax) pm[i & 3] = fmaxf(pm[i & 3], fmaxf(x0, x1));
-            const float p0 = ex2_approx(fmaf(x0, c, neg_m));
-            const float p1 = ex2_approx(fmaf(x1, c, neg_m));
-            ps[i & 3] += p0 + p1;
-            pk[i] = pack_bf16x2(p0, p1);
-        }
-        tmem_st_x16(tS + 16 * q2, pk);
+        for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+        tmem_st_x32(tO + 32u * cc, o);
     }
-    if (hmax) *hmax = fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3]));
-    return (ps[0] + ps[1]) + (ps[2] + ps[3]);
 }
 
-// Softmax of query tile t, key columns [64*hf, 64*hf + 64) of every 128-key
-// block: thread r owns row r (TMEM lane r) of that half.  The two halves of a
-// row run in two warpgroups and agree on the row's reference max through
-// shared memory and a bounded mbarrier wait per block.
+// Softmax of query tile t: thread r owns row r (TMEM lane r), all 128 keys.
 template <int D>
-__device__ void softmax_group(AttnSmem<D>& sm, const AttnArgs& a, uint32_t tmem, int t, int hf, int b, int h, int qb,
+__device__ void softmax_group(AttnSmem<D>& sm, const AttnArgs& a, uint32_t tmem, int t, int b, int h, int qb,
                               const int32_t* list, volatile int* abort_flag) {
     const int lane = threadIdx.x & 31;
     const int quarter = (threadIdx.x >> 5) & 3;  // TMEM lanes [32*quarter, 32*quarter + 32)
     const int row = quarter * 32 + lane;
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
-    const uint32_t tS = tmem + lane_addr + col_s(t) + 64u * hf;
-    const uint32_t tO = tmem + lane_addr + Geo<D>::col_o(t) + static_cast<uint32_t>(Geo<D>::kHalf) * hf;
-    constexpr int kRest = Geo<D>::kHalf - 32;  // O columns of the half beyond the first 32 (16 or 32)
+    const uint32_t tS = tmem + lane_addr + col_s(t);
+    const uint32_t tO = tmem + lane_addr + Geo<D>::col_o(t);
     const float c = a.scale_log2;
     float m_used = -INFINITY;  // row reference max of scaled logits (log2 units)
-    float l = 0.f;             // this half's running sum of P
+    float l = 0.f;             // running row sum of P
     bool ok = true;
     for (int j = 0; j < a.n_iter; ++j) {
         // warp-uniform outcome: the tcgen05.ld/st below are warp-collective
@@ -371,80 +348,56 @@ __device__ void softmax_group(AttnSmem<D>& sm, const AttnArgs& a, uint32_t tmem,
             break;
         }
         tc_fence_after_sync();
-        uint32_t s[2][32];
-        tmem_ld_x32(tS + 0, s[0]);
-        tmem_ld_x32(tS + 32, s[1]);
-        tmem_wait_ld_x32(s[0]);
-        tmem_wait_ld_x32(s[1]);
-
         const int kv = list ? __ldg(list + j) : j;
-        const int valid = (kv == a.nblk - 1) ? a.N - kv * 128 - 64 * hf : 64;
-        if (valid < 64) {
+        const int valid = (kv == a.nblk - 1) ? a.N - kv * 128 : 128;
+        // the whole row of S in registers: one wait, the true block max before
+        // any exponential, P packed in place over the same registers
+        uint32_t x[128];
 #pragma unroll
-            for (int q2 = 0; q2 < 2; ++q2)
+        for (int q = 0; q < 4; ++q) tmem_ld_x32(tS + 32u * q, slice32(x + 32 * q));
 #pragma unroll
-                for (int i = 0; i < 32; ++i)
-                    if (q2 * 32 + i >= valid) s[q2][i] = __float_as_uint(-INFINITY);
+        for (int q = 0; q < 4; ++q) tmem_wait_ld_x32(slice32(x + 32 * q));
+        if (valid < 128) {
+#pragma unroll
+            for (int i = 0; i < 128; ++i)
+                if (i >= valid) x[i] = __float_as_uint(-INFINITY);
         }
-        float hm;
-        float* xm = &sm.xmax[j & 1][t][0][0];
-        uint64_t* xb = &sm.xbar[j & 1][t];
-        const uint32_t xpar = static_cast<uint32_t>((j >> 1) & 1);
+        float pm[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+        for (int i = 0; i < 64; ++i)
+            pm[i & 3] = max3(pm[i & 3], __uint_as_float(x[2 * i]), __uint_as_float(x[2 * i + 1]));
+        const float mx = c * fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3]));
         if (j == 0) {
-            // the first block fixes the reference: exchange half maxima before the exponentials
-            float pm[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-            for (int q2 = 0; q2 < 2; ++q2)
-#pragma unroll
-                for (int i = 0; i < 32; ++i) pm[i & 3] = fmaxf(pm[i & 3], __uint_as_float(s[q2][i]));
-            hm = fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3]));
-            xm[hf * 128 + row] = hm;
-            __syncwarp();
-            if (lane == 0) mbar_arrive(xb);
-            if (!__all_sync(0xffffffffu, mbar_wait(xb, xpar, abort_flag, a.timeout_ns))) {
-                ok = false;
-                break;
-            }
-            m_used = c * fmaxf(hm, xm[(hf ^ 1) * 128 + row]);
-            l += exp_store_half(s, c, m_used, tS, nullptr);
+            m_used = mx;  // the first block fixes the reference
         } else {
-            // later blocks start with the running reference (stale by design) and
-            // check the block max afterwards; only a row whose max grew by more than
-            // 2^8 recomputes its P and rescales O and its sum -- the final division
-            // by the row sum keeps the result exact either way
-            const float ps = exp_store_half(s, c, m_used, tS, &hm);
-            xm[hf * 128 + row] = hm;
-            __syncwarp();
-            if (lane == 0) mbar_arrive(xb);
-            if (!__all_sync(0xffffffffu, mbar_wait(xb, xpar, abort_flag, a.timeout_ns))) {
-                ok = false;
-                break;
-            }
-            const float mx = c * fmaxf(hm, xm[(hf ^ 1) * 128 + row]);
             const bool need = mx - m_used > 8.0f;
             if (__any_sync(0xffffffffu, need)) {
-                // O_t is stable here: the commit behind s_full covers PV(j-1)
+                // rare: O_t is stable here (the commit behind s_full covers PV_t(j-1))
                 float alpha = 1.0f;
                 if (need) {
                     alpha = ex2_approx(m_used - mx);
                     m_used = mx;
                 }
-                l = l * alpha + exp_store_half(s, c, m_used, tS, nullptr);
-                uint32_t o[32], o2[kRest];
-                tmem_ld_x32(tO, o);
-                tmem_ld_n(tO + 32, o2);
-                tmem_wait_ld_x32(o);
-                tmem_wait_ld_n(o2);
-#pragma unroll
-                for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-#pragma unroll
-                for (int i = 0; i < kRest; ++i) o2[i] = __float_as_uint(__uint_as_float(o2[i]) * alpha);
-                tmem_st_x32(tO, o);
-                tmem_st_n(tO + 32, o2);
-            } else {
-                l += ps;
+                l *= alpha;
+                rescale_o<D>(tO, alpha);
             }
         }
+        const uint64_t c2 = f2(c, c), nm2 = f2(-m_used, -m_used);
+        uint64_t acc[2] = {f2(0.f, 0.f), f2(0.f, 0.f)};
+#pragma unroll
+        for (int i = 0; i < 64; ++i) {
+            float a0, a1;
+            f2_split(f2_fma(f2(__uint_as_float(x[2 * i]), __uint_as_float(x[2 * i + 1])), c2, nm2), a0, a1);
+            const float p0 = ex2_approx(a0), p1 = ex2_approx(a1);
+            acc[i & 1] = f2_add(acc[i & 1], f2(p0, p1));
+            x[i] = pack_bf16x2(p0, p1);  // i < 2i: the S values read here are never needed again
+        }
+        float s0, s1, s2, s3;
+        f2_split(acc[0], s0, s1);
+        f2_split(acc[1], s2, s3);
+        l += (s0 + s1) + (s2 + s3);
+        tmem_st_x32(tS, slice32(x));
+        tmem_st_x32(tS + 32, slice32(x + 32));
         // one arrival per warp: every lane's TMEM stores are complete and
         // fenced before the warp converges and lane 0 releases the barrier
         tmem_wait_st();
@@ -456,37 +409,29 @@ __device__ void softmax_group(AttnSmem<D>& sm, const AttnArgs& a, uint32_t tmem,
         raise_timeout(a, abort_flag);
         return;
     }
-    // row sum = both halves
-    sm.lsum[t][hf][row] = l;
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&sm.lbar[t]);
-    if (!__all_sync(0xffffffffu, mbar_wait(&sm.lbar[t], 0u, abort_flag, a.timeout_ns)) ||
-        !__all_sync(0xffffffffu, mbar_wait(&sm.o_done[t], 0u, abort_flag, a.timeout_ns))) {
+    if (!__all_sync(0xffffffffu, mbar_wait(&sm.o_done[t], 0u, abort_flag, a.timeout_ns))) {
         raise_timeout(a, abort_flag);
         return;
     }
     tc_fence_after_sync();
-    const float inv_l = 1.0f / (l + sm.lsum[t][hf ^ 1][row]);
+    const float inv_l = 1.0f / l;
     const int n = qb * 128 + row;
-    uint32_t o[32], o2[kRest];
-    tmem_ld_x32(tO, o);
-    tmem_ld_n(tO + 32, o2);
-    tmem_wait_ld_x32(o);
-    tmem_wait_ld_n(o2);
-    if (n < a.N) {
-        __nv_bfloat16* dst = a.o + static_cast<int64_t>(b) * a.sb + static_cast<int64_t>(n) * a.sn +
-                             static_cast<int64_t>(h) * a.sh + Geo<D>::kHalf * hf;
-        uint32_t w[Geo<D>::kHalf / 2];
+    __nv_bfloat16* dst = a.o + static_cast<int64_t>(b) * a.sb + static_cast<int64_t>(n) * a.sn +
+                         static_cast<int64_t>(h) * a.sh;
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-            w[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
+    for (int cc = 0; cc < Geo<D>::kChunks; ++cc) {
+        uint32_t o[32];
+        tmem_ld_x32(tO + 32u * cc, o);
+        tmem_wait_ld_x32(o);
+        if (n < a.N) {
+            uint32_t w[16];
 #pragma unroll
-        for (int i = 0; i < kRest / 2; ++i)
-            w[16 + i] = pack_bf16x2(__uint_as_float(o2[2 * i]) * inv_l, __uint_as_float(o2[2 * i + 1]) * inv_l);
-        uint4* d4 = reinterpret_cast<uint4*>(dst);
+            for (int i = 0; i < 16; ++i)
+                w[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
+            uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * cc);
 #pragma unroll
-        for (int i = 0; i < Geo<D>::kHalf / 8; ++i)
-            d4[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+            for (int i = 0; i < 4; ++i) d4[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+        }
     }
 }
 
@@ -511,10 +456,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int t = 0; t < 2; ++t) {
             mbar_init(&sm.q_full[t], 1);
             mbar_init(&sm.s_full[t], 1);
-            mbar_init(&sm.p_full[t], 8);  // one arrival per softmax warp of the tile
-            mbar_init(&sm.xbar[0][t], 8);
-            mbar_init(&sm.xbar[1][t], 8);
-            mbar_init(&sm.lbar[t], 8);
+            mbar_init(&sm.p_full[t], 4);  // one arrival per softmax warp of the tile
             mbar_init(&sm.o_done[t], 1);
         }
         for (int s = 0; s < Geo<D>::kStages; ++s) {
@@ -543,9 +485,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == kMmaWarp) {
         if ((threadIdx.x & 31) == 0) mma_issuer<D>(sm, a, tmem, has1, l0, l1, abort_flag);
     } else {
-        const int wg = warp >> 2;  // softmax warpgroup: tile wg / 2, column half wg % 2
-        const int t = wg >> 1, hf = wg & 1;
-        if (t == 0 || has1) softmax_group<D>(sm, a, tmem, t, hf, b, h, qb0 + t, t ? l1 : l0, abort_flag);
+        const int t = warp >> 2;  // softmax warpgroup = query tile
+        if (t == 0 || has1) softmax_group<D>(sm, a, tmem, t, b, h, qb0 + t, t ? l1 : l0, abort_flag);
     }
     tc_fence_before_sync();
     __syncthreads();

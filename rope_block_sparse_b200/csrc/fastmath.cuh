@@ -1,5 +1,5 @@
-// Packed fp32 pair arithmetic (f32x2 instructions of sm_100a) and the
-// FMA-pipe exp2 used by the attention softmax.
+// Packed fp32 pair arithmetic (f32x2 instructions of sm_100a) used by the
+// attention softmax, a three-input max, and an FMA-pipe exp2 (self-test only).
 #pragma once
 
 #include <cstdint>
@@ -30,6 +30,13 @@ __device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
     asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
     return r;
 }
+// max(a, b, c) in one instruction (three-input max.f32 of sm_100a).
+__device__ __forceinline__ float max3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
 // 2^x for a pair on the FMA pipe instead of the MUFU unit: x = n + f with
 // n = round(x) (adding 1.5 * 2^23 leaves n in the low mantissa bits) and
 // f in [-1/2, 1/2]; 2^f from a degree-3 polynomial minimising the relative
