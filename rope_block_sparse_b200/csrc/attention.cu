@@ -9,7 +9,7 @@
 // 2p and 2p+1, i.e. the router's query blocks -- and streams 128-row K/V tiles
 // through shared memory: every KV block for dense attention, or each tile's
 // own routed list in sparse mode (a KV tile both lists name at the same step is
-// loaded once and shared).  Warp roles (320 threads, 10 warps):
+// loaded once and shared).  Warp roles (384 threads, 12 warps):
 //   warps 0-7   softmax: warpgroup t = warp / 4 handles query tile t; thread r
 //               owns row r (TMEM lane r) and all 128 key columns of every
 //               block, so the row max and row sum never leave the thread.  It
@@ -30,6 +30,8 @@
 //               TMEM, V as an MN-major operand).  Order per step j:
 //               PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1), so each softmax group
 //               waits only on its own tile's chain.
+//   warps 10-11 idle: they complete the third warpgroup, whose registers
+//               (setmaxnreg) go to the softmax warpgroups (200 each).
 // TMEM columns: S_0 [0,128), S_1 [128,256), O_0 [256,352), O_1 [352,448) at
 // head_dim 96; the same kernel is instantiated for head_dim 128 (O_0
 // [256,384), O_1 [384,512), four 32-channel chunks per tile, 2-stage rings).
@@ -46,7 +48,15 @@ namespace {
 
 constexpr int kSoftmaxWarps = 8;                   // 2 warpgroups: one per query tile
 constexpr int kProducerWarp = 8, kMmaWarp = 9;
-constexpr int kThreads = 32 * (kSoftmaxWarps + 2);  // 320
+constexpr int kThreads = 32 * (kSoftmaxWarps + 4);  // 384: warps 10-11 idle (a full third warpgroup)
+// Register split (setmaxnreg, per warpgroup): the launch gives every thread
+// 168 registers (65,536 / 384 rounded down to 8); the third warpgroup
+// (producer, MMA issuer, two idle warps) drops to 80 and the two softmax
+// warpgroups rise to 200, so a softmax thread holds its 128-value row without
+// spilling.  The new total must fit in what the block was launched with.
+constexpr uint32_t kRegsLaunch = (65536 / kThreads) / 8 * 8;
+constexpr uint32_t kRegsSoftmax = 200, kRegsOther = 80;
+static_assert(kSoftmaxWarps * 32 * kRegsSoftmax + 128 * kRegsOther <= kThreads * kRegsLaunch, "register split");
 constexpr int kChunkBytes = 128 * 64;        // 128 rows x 32 bf16, 64-byte swizzle
 constexpr uint32_t kTmemCols = 512;
 // TMEM column of S_t
@@ -480,13 +490,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem = sm.tmem_base;
     volatile int* abort_flag = &sm.abort_flag;
 
-    if (warp == kProducerWarp) {
-        if ((threadIdx.x & 31) == 0) producer<D>(sm, a, &tq, &tk, &tv, b, h, qb0, has1, l0, l1, abort_flag);
-    } else if (warp == kMmaWarp) {
-        if ((threadIdx.x & 31) == 0) mma_issuer<D>(sm, a, tmem, has1, l0, l1, abort_flag);
-    } else {
+    if (warp < kSoftmaxWarps) {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
         const int t = warp >> 2;  // softmax warpgroup = query tile
         if (t == 0 || has1) softmax_group<D>(sm, a, tmem, t, b, h, qb0 + t, t ? l1 : l0, abort_flag);
+    } else {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsOther));
+        if (warp == kProducerWarp) {
+            if ((threadIdx.x & 31) == 0) producer<D>(sm, a, &tq, &tk, &tv, b, h, qb0, has1, l0, l1, abort_flag);
+        } else if (warp == kMmaWarp) {
+            if ((threadIdx.x & 31) == 0) mma_issuer<D>(sm, a, tmem, has1, l0, l1, abort_flag);
+        }
     }
     tc_fence_before_sync();
     __syncthreads();
