@@ -17,11 +17,12 @@
 //               block max, computes exp2 in fp32 (log2 domain, packed f32x2
 //               FMAs and adds) against the row's reference max, packs P to bf16
 //               in place over the same registers and writes it over the first
-//               64 columns of S.  The reference is fixed by the first block; a
-//               later block moves it up and rescales O (in TMEM) only when the
-//               row max grew by more than 2^8 (the final division by the row
-//               sum keeps this exact).  At the end the thread divides its O row
-//               by the row sum, rounds once to bf16 and stores it.
+//               64 columns of S, each 16-column chunk as soon as it is
+//               complete.  The reference is fixed by the first block; a later
+//               block moves it up and rescales O (in TMEM) only when the row
+//               max grew by more than 2^8 (the final division by the row sum
+//               keeps this exact).  At the end the thread divides its O row by
+//               the row sum, rounds once to bf16 and stores it.
 //   warp 8      TMA producer: Q tiles once, then a 3-stage K ring and a 3-stage
 //               V ring (64-byte swizzled 128 x 32 chunks, 3 per 128 x 96 tile).
 //   warp 9      owns tensor memory (512 columns) and issues tcgen05.mma from one
@@ -321,6 +322,7 @@ __device__ void mma_issuer(AttnSmem<D>& sm, const AttnArgs& a, uint32_t tmem, bo
 
 // tcgen05.ld of 32 columns into / wait on a 32-register slice of a longer row.
 __device__ __forceinline__ uint32_t (&slice32(uint32_t* x))[32] { return *reinterpret_cast<uint32_t(*)[32]>(x); }
+__device__ __forceinline__ uint32_t (&slice16(uint32_t* x))[16] { return *reinterpret_cast<uint32_t(*)[16]>(x); }
 
 // O row *= alpha (rare rescale).  Out of line: it runs only when a row max
 // grows by more than 2^8, and its registers stay out of the steady-state loop.
@@ -361,7 +363,9 @@ __device__ void softmax_group(AttnSmem<D>& sm, const AttnArgs& a, uint32_t tmem,
         const int kv = list ? __ldg(list + j) : j;
         const int valid = (kv == a.nblk - 1) ? a.N - kv * 128 : 128;
         // the whole row of S in registers: one wait, the true block max before
-        // any exponential, P packed in place over the same registers
+        // any exponential, P packed in place over the same registers and
+        // stored in 16-column chunks as they complete (over S columns already
+        // read), so little store traffic is left to wait for at the end
         uint32_t x[128];
 #pragma unroll
         for (int q = 0; q < 4; ++q) tmem_ld_x32(tS + 32u * q, slice32(x + 32 * q));
@@ -401,13 +405,12 @@ __device__ void softmax_group(AttnSmem<D>& sm, const AttnArgs& a, uint32_t tmem,
             const float p0 = ex2_approx(a0), p1 = ex2_approx(a1);
             acc[i & 1] = f2_add(acc[i & 1], f2(p0, p1));
             x[i] = pack_bf16x2(p0, p1);  // i < 2i: the S values read here are never needed again
+            if ((i & 15) == 15) tmem_st_x16(tS + (i - 15), slice16(x + (i - 15)));
         }
         float s0, s1, s2, s3;
         f2_split(acc[0], s0, s1);
         f2_split(acc[1], s2, s3);
         l += (s0 + s1) + (s2 + s3);
-        tmem_st_x32(tS, slice32(x));
-        tmem_st_x32(tS + 32, slice32(x + 32));
         // one arrival per warp: every lane's TMEM stores are complete and
         // fenced before the warp converges and lane 0 releases the barrier
         tmem_wait_st();
