@@ -121,3 +121,19 @@ def test_layer8k_42_heads_sampled_d128(orc):
     check_attention(gather_rows(o_dense, rows), orc.attention_rows(d["q"], d["k"], d["v"], rows), "d128 dense")
     check_attention(gather_rows(o_sparse, rows), orc.attention_rows(d["q"], d["k"], d["v"], rows, ora_idx),
                     "d128 sparse")
+
+
+def test_reference_moves_up_d128(orc):
+    """Key blocks scaled 0.05, 1, 4, 0.05, 16, 32 (the last one a tail of 16
+    keys): most rows move their reference max up at blocks 2 and 4 and two in
+    three at the tail, so O (128 columns here) is rescaled in TMEM mid-row."""
+    grid, heads = (2, 8, 41), 2                   # 656 tokens, 6 blocks
+    d = _inputs(1, heads, grid, seed=5)
+    f = torch.tensor([0.05, 1.0, 4.0, 0.05, 16.0, 32.0]).repeat_interleave(128)[:656]
+    d["k"] = (d["k"].float() * f[None, :, None, None]).to(torch.bfloat16)
+    d["v"] = (d["v"].float() * 0.25).to(torch.bfloat16)   # |O| < 2: one bf16 ulp well inside 2e-2
+    o = h3a.attention(_dev(d["q"]), _dev(d["k"]), _dev(d["v"]))
+    torch.cuda.synchronize()
+    assert h3a.last_device_error() == 0
+    rows = np.arange(heads * 656)
+    check_attention(gather_rows(o, rows), orc.attention_rows(d["q"], d["k"], d["v"], rows), "d128 growing keys")

@@ -189,6 +189,53 @@ def test_identical_keys_give_mean_value():
     assert err <= 2e-3, err
 
 
+def _growing_keys(heads, grid, scales, seed=5):
+    """Seeded inputs whose key block b is scaled by scales[b]: the logits of a
+    later block outgrow the reference max fixed by the first block -- by far
+    more than 2^8 in the log2 domain for most rows of blocks 2, 4 and the
+    ragged tail, by less for others -- so the kernel must move its reference
+    up and rescale O and the row sum, in some rows of a warp and not others."""
+    d = _inputs(1, heads, grid, "normal", seed)
+    N = grid[0] * grid[1] * grid[2]
+    assert len(scales) == (N + 127) // 128
+    f = torch.tensor(scales, dtype=torch.float32).repeat_interleave(128)[:N]
+    d["k"] = (d["k"].float() * f[None, :, None, None]).to(torch.bfloat16)
+    # a few keys dominate each row, so O is close to single rows of V: V is
+    # scaled down to keep |O| < 2, where one bf16 ulp of the output stays well
+    # inside the 2e-2 bound
+    d["v"] = (d["v"].float() * 0.25).to(torch.bfloat16)
+    return d
+
+
+GROWING = [0.05, 1.0, 4.0, 0.05, 16.0, 32.0]     # 6 blocks: 5 full + a tail of 16 keys
+
+
+def test_attention_reference_moves_up_dense(orc):
+    grid, heads = (2, 8, 41), 3                  # 656 tokens
+    d = _growing_keys(heads, grid, GROWING)
+    o = h3a.attention(_dev(d["q"]), _dev(d["k"]), _dev(d["v"]))
+    torch.cuda.synchronize()
+    assert h3a.last_device_error() == 0
+    rows = np.arange(heads * 656)
+    want = orc.attention_rows(d["q"], d["k"], d["v"], rows)
+    check_attention(gather_rows(o, rows), want, "growing keys, dense")
+
+
+def test_attention_reference_moves_up_sparse(orc):
+    """Hand-made ascending lists: a small block first and larger ones after,
+    a large block first with a small one after it, the tail block last."""
+    grid, heads = (2, 8, 41), 2
+    d = _growing_keys(heads, grid, GROWING, seed=6)
+    lists = [[0, 2, 3, 5], [2, 3, 4, 5], [0, 1, 2, 4], [1, 3, 4, 5], [0, 3, 4, 5], [1, 2, 4, 5]]
+    idx = np.array(lists, dtype=np.int32)[None, None].repeat(heads, axis=1)   # [1, heads, 6, 4]
+    o = h3a.attention(_dev(d["q"]), _dev(d["k"]), _dev(d["v"]), _dev(torch.from_numpy(np.ascontiguousarray(idx))))
+    torch.cuda.synchronize()
+    assert h3a.last_device_error() == 0
+    rows = np.arange(heads * 656)
+    want = orc.attention_rows(d["q"], d["k"], d["v"], rows, idx)
+    check_attention(gather_rows(o, rows), want, "growing keys, sparse")
+
+
 def test_dense_attention_layer8k_sampled(orc):
     d = synth.draw_workload("layer8k")
     o = h3a.attention(_dev(d["q"]), _dev(d["k"]), _dev(d["v"]))
