@@ -189,6 +189,71 @@ def test_identical_keys_give_mean_value():
     assert err <= 2e-3, err
 
 
+def test_chain_head_major_storage(orc):
+    """Q, K, V and every output stored head-major ([B, heads, N, 96] memory
+    viewed as [B, N, heads, 96]: token stride 96, head stride N*96) through
+    the prologue, the router and dense and sparse attention, each stage
+    against the oracle on the previous stage's GPU output."""
+    grid, heads = (3, 8, 25), 3                   # 600 tokens, 5 blocks
+    d = _inputs(1, heads, grid, "structured", 8)
+    hm = {n: _dev(d[n].transpose(1, 2).contiguous()).transpose(1, 2) for n in "qkv"}
+    assert hm["q"].stride() == (heads * 600 * 96, 96, 600 * 96, 1)
+    qn, kn = h3a.qk_norm_rope(hm["q"], hm["k"], _dev(d["gamma_q"]), _dev(d["gamma_k"]), grid, THETA, EPS)
+    idx = h3a.route(qn, kn, 0.6)
+    dense = h3a.attention(qn, kn, hm["v"])
+    sparse = h3a.attention(qn, kn, hm["v"], idx)
+    torch.cuda.synchronize()
+    assert h3a.last_device_error() == 0
+    assert qn.stride() == dense.stride() == sparse.stride() == hm["q"].stride()
+    for x, g, out in ((d["q"], d["gamma_q"], qn), (d["k"], d["gamma_k"], kn)):
+        check_prologue(bits(out), orc.qk_norm_rope_bf16(x, g.numpy(), grid, THETA, EPS), "head-major")
+    qb, kb = bits(qn), bits(kn)
+    ora_idx, ora_sc = orc.route(qb, kb, 0.6)
+    gpu_idx = idx.cpu().numpy()
+    check_router(gpu_idx, ora_idx, ora_sc, "head-major")
+    rows = np.arange(heads * 600)
+    check_attention(gather_rows(dense, rows), orc.attention_rows(qb, kb, d["v"], rows), "head-major dense")
+    check_attention(gather_rows(sparse, rows), orc.attention_rows(qb, kb, d["v"], rows, gpu_idx),
+                    "head-major sparse")
+
+
+def test_attention_heads_of_a_wider_buffer(orc):
+    """Heads 2..6 of a 9-head buffer (token stride 9*96, offset 2*96), output
+    written into the same columns of another 9-head buffer; the rest untouched."""
+    grid, heads = (2, 8, 20), 9                   # 320 tokens, 3 blocks
+    d = _inputs(1, heads, grid, "normal", 9)
+    q, k, v = (_dev(d[n])[:, :, 2:7] for n in "qkv")
+    obuf = torch.full((1, 320, heads, 96), 7.0, dtype=torch.bfloat16, device="cuda")
+    o = obuf[:, :, 2:7]
+    h3a.attention(q, k, v, out=o)
+    torch.cuda.synchronize()
+    assert h3a.last_device_error() == 0
+    assert bool((obuf[:, :, :2] == 7.0).all()) and bool((obuf[:, :, 7:] == 7.0).all())
+    sub = {n: d[n][:, :, 2:7].contiguous() for n in "qkv"}
+    rows = np.arange(5 * 320)
+    check_attention(gather_rows(o, rows), orc.attention_rows(sub["q"], sub["k"], sub["v"], rows), "head slice")
+
+
+@pytest.mark.parametrize("scale", [0.02, 0.4])
+def test_attention_explicit_scale(orc, scale):
+    """A caller-given logit scale instead of 1/sqrt(96): nearly uniform weights
+    at 0.02, sharp rows (reference moved up often) at 0.4; dense and sparse."""
+    grid, heads = (2, 8, 30), 2                   # 480 tokens, 4 blocks (tail of 96)
+    d = _inputs(1, heads, grid, "structured", 10)
+    d["v"] = (d["v"].float() * 0.25).to(torch.bfloat16)   # sharp rows: keep |O| < 2
+    q, k, v = (_dev(d[n]) for n in "qkv")
+    ora_idx, _ = orc.route(d["q"], d["k"], 0.5)
+    dense = h3a.attention(q, k, v, scale=scale)
+    sparse = h3a.attention(q, k, v, _dev(torch.from_numpy(ora_idx)), scale=scale)
+    torch.cuda.synchronize()
+    assert h3a.last_device_error() == 0
+    rows = np.arange(heads * 480)
+    check_attention(gather_rows(dense, rows), orc.attention_rows(d["q"], d["k"], d["v"], rows, scale=scale),
+                    f"scale {scale} dense")
+    check_attention(gather_rows(sparse, rows),
+                    orc.attention_rows(d["q"], d["k"], d["v"], rows, ora_idx, scale=scale), f"scale {scale} sparse")
+
+
 def _growing_keys(heads, grid, scales, seed=5):
     """Seeded inputs whose key block b is scaled by scales[b]: the logits of a
     later block outgrow the reference max fixed by the first block -- by far
