@@ -6,8 +6,8 @@
 // the CUDA library; both sides only receive the same seeded input arrays.
 //
 // What it states, each function citing the passage it follows:
-//   * QK-RMSNorm followed by 3D RoPE, fused and lossless ("changes no computed
-//     result"): news.cocoloop.cn, MiniMax-H3 SGLang report, section "Erst drei
+//   * QK-RMSNorm followed by 3D RoPE, fused and lossless (the fusion leaves the
+//     results unchanged): news.cocoloop.cn, MiniMax-H3 SGLang report, section "Erst drei
 //     übereinandergelegte Beschleunigungsebenen", fused-operator paragraph.
 //     The 3D multimodal RoPE and the head geometry (hidden 5376 / 56 heads = 96)
 //     come from 52hbtv.com, H3-Image port, section 二, model table.
@@ -15,8 +15,8 @@
 //     SubBlock paragraph); pooling, scoring and selection are fixed by the
 //     problem statement: mean-pooled 128-token blocks, fp32 block scores,
 //     per-query-block top-k, ties to the lower block index.
-//   * Dense lossless attention (cocoloop page, opening quote: "no
-//     approximation") and block-sparse attention over the routed KV blocks,
+//   * Dense lossless attention (cocoloop page, opening quote: the dense path
+//     approximates nothing) and block-sparse attention over the routed KV blocks,
 //     bidirectional (cocoloop page, "Ein paar Grenzen": non-causal).
 //   * The other operators the fused-operator paragraph of the cocoloop page
 //     names -- the AdaLN update, the gated residual path and the SwiGLU
