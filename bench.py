@@ -34,6 +34,7 @@ sys.path.insert(0, ROOT)
 WORKLOAD = "video5s_sparse"
 FFN_WIDTH = 14336  # DiT FFN width of the model table (52hbtv.com H3-Image page, section 二)
 SPARSITY = 0.75
+L2_GB = 0.126  # B200 L2: 126 MB
 METRIC = "attention TFLOP/s and % of B200 bf16 peak at ~125k tokens; prologue GB/s vs HBM"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
@@ -183,6 +184,25 @@ def load_traffic():
         if h.hexdigest() == ent["sha256"]:
             out[kernel] = ent
     return out
+
+
+def config_of(w, world: int, kk: int) -> dict:
+    """The workload description both arms print (kk: KV blocks kept per query block)."""
+    B, N, heads, D, grid = w.B, w.N, w.heads, w.head_dim, w.grid
+    nblk = (N + 127) // 128
+    wide = D != 96
+    gb = B * N * heads * D * 2 / 1e9
+    return {
+        "workload": f"{w.name}: B={B}, {heads} heads x {D}, grid {grid[0]}x{grid[1]}x{grid[2]} = {N:,} tokens "
+                    f"per GPU; " + (f"router with its own pooling (sparsity {SPARSITY}, k={kk}/{nblk}) + sparse + "
+                                    "dense attention (no prologue: its 3D RoPE is defined for 96 channels)" if wide
+                                    else f"prologue with block pooling + router scores/top-k (sparsity {SPARSITY}, "
+                                    f"k={kk}/{nblk}) + sparse + dense attention"),
+        "tokens": N, "heads": heads, "head_dim": D, "batch_per_gpu": B, "sparsity": SPARSITY,
+        "parallelism": f"dp{world} (independent clips per GPU)",
+        "l2": (f"inputs larger than L2 (Q, K, V {gb:.2f} GB each); no explicit flush" if 3 * gb > L2_GB
+               else f"inputs fit in L2 (Q, K, V {gb * 1e3:.2f} MB each): a correctness-size case, not a timing one"),
+    }
 
 
 # ----------------------------------------------------------------- GPU arm
@@ -400,16 +420,7 @@ def run_gpu(args, rank, world, local):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic",
-        "config": {
-            "workload": f"{w.name}: B={B}, {heads} heads x {D}, grid {grid[0]}x{grid[1]}x{grid[2]} = {N:,} tokens "
-                        f"per GPU; " + (f"router with its own pooling (sparsity {SPARSITY}, k={kk}/{nblk}) + sparse + "
-                                        "dense attention (no prologue: its 3D RoPE is defined for 96 channels)" if wide
-                                        else f"prologue with block pooling + router scores/top-k (sparsity {SPARSITY}, "
-                                        f"k={kk}/{nblk}) + sparse + dense attention"),
-            "tokens": N, "heads": heads, "head_dim": D, "batch_per_gpu": B, "sparsity": SPARSITY,
-            "parallelism": f"dp{world} (independent clips per GPU)",
-            "l2": f"inputs larger than L2 (Q, K, V {B * N * heads * D * 2 / 1e9:.2f} GB each); no explicit flush",
-        },
+        "config": config_of(w, world, kk),
         "roofline": {
             "kernel": "attention_kernel (dense)",
             "bound": "tensor",
@@ -567,10 +578,10 @@ def run_reference(args, rank, world):
     import oracle
     from rope_block_sparse_b200 import synth
 
-    w = synth.WORKLOADS[WORKLOAD]
-    d = synth.draw_workload(WORKLOAD, seed=0)
+    w = synth.WORKLOADS[args.workload]
+    d = synth.draw_workload(args.workload, seed=0)
     qb, kb, idx = _oracle_inputs(d, w, SPARSITY)
-    rows_per_step = args.ref_rows
+    rows_per_step = min(args.ref_rows, w.B * w.heads * w.N)
     times, flops = [], []
     for i in range(args.warmup + args.steps):
         rows = synth.sample_rows(w.B, w.heads, w.N, rows_per_step, seed=1000 + i).numpy()
@@ -579,8 +590,8 @@ def run_reference(args, rank, world):
             times.append(dt)
             flops.append(fl)
     value = sum(flops) / sum(times) / 1e12
-    sample = (f"fp64 oracle dense + sparse (0.75) attention for {rows_per_step} sampled query rows per step of "
-              f"{WORKLOAD}; prologue and router outputs precomputed by the oracle")
+    sample = (f"fp64 oracle dense + sparse ({SPARSITY}) attention for {rows_per_step} sampled query rows per step "
+              f"of {w.name}; prologue and router outputs precomputed by the oracle")
     return {
         "impl": "reference",
         "metric": METRIC,
@@ -595,8 +606,7 @@ def run_reference(args, rank, world):
         "vs_baseline": None,
         "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": f"{WORKLOAD}: B=1, 56 heads x 96, grid 31x48x84 = 124,992 tokens",
-                   "tokens": w.N, "heads": w.heads, "sparsity": SPARSITY},
+        "config": config_of(w, world, idx.shape[-1]),
         "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": oracle.threads(), "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
