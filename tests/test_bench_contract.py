@@ -48,3 +48,25 @@ def test_config_names_the_workload_not_a_model():
     assert "k=245/977" in c["workload"] and c["parallelism"].startswith("dp8")
     assert c["tokens"] == 124992 and c["heads"] == 56 and c["head_dim"] == 96 and c["sparsity"] == bench.SPARSITY
     assert c["l2"].startswith("inputs larger than L2")
+
+
+def _free_port() -> int:
+    import socket
+
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def test_reference_arm_under_torchrun_prints_once():
+    """Two ranks launched the way the multi-GPU bench is: rank 0 alone runs the
+    oracle and prints; the other rank exits 0 without work."""
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(_free_port()), "bench.py", "--impl", "reference",
+           "--gpus", "2", "--workload", "tiny", "--steps", "1", "--warmup", "3", "--ref-rows", "8"]
+    res = subprocess.run(cmd, cwd=ROOT, capture_output=True, text=True, timeout=600)
+    assert res.returncode == 0, res.stderr[-2000:]
+    lines = [ln for ln in res.stdout.splitlines() if ln.strip().startswith("{")]
+    assert len(lines) == 1, res.stdout
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["config"]["parallelism"].startswith("dp2")
