@@ -15,29 +15,33 @@
 //               block, so the row max and row sum never leave the thread.  It
 //               loads the whole row of S from TMEM with one wait, takes the
 //               block max, computes exp2 in fp32 (log2 domain, packed f32x2
-//               FMAs and adds) against the row's reference max, packs P to bf16
-//               in place over the same registers and writes it over the first
-//               64 columns of S, each 16-column chunk as soon as it is
-//               complete.  The reference is fixed by the first block; a later
-//               block moves it up and rescales O (in TMEM) only when the row
-//               max grew by more than 2^8 (the final division by the row sum
-//               keeps this exact).  At the end the thread divides its O row by
-//               the row sum, rounds once to bf16 and stores it.
-//   warp 8      TMA producer: Q tiles once, then a 3-stage K ring and a 3-stage
-//               V ring (64-byte swizzled 128 x 32 chunks, 3 per 128 x 96 tile).
-//   warp 9      owns tensor memory (512 columns) and issues tcgen05.mma from one
-//               thread: S_t = Q_t K^T (M=128, N=128, K=96 as 6 steps of 16) into
-//               TMEM, O_t += P_t V (M=128, N=96, K=128 as 8 steps, P read from
-//               TMEM, V as an MN-major operand).  Order per step j:
-//               PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1), so each softmax group
-//               waits only on its own tile's chain.
-//   warps 10-11 idle: they complete the third warpgroup, whose registers
+//               FMAs and adds) against the row's reference max and packs P to
+//               bf16 in place over the same registers.  The reference is fixed
+//               by the first block; a later block moves it up and rescales O
+//               (in TMEM) only when the row max grew by more than 2^8 (the
+//               final division by the row sum keeps this exact).  At the end
+//               the thread divides its O row by the row sum, rounds once to
+//               bf16 and stores it.
+//   warp 8      TMA producer: Q tiles once, then a K ring and a V ring
+//               (64-byte swizzled 128 x 32 chunks, D/32 per 128 x D tile).
+//   warp 9      owns tensor memory (512 columns) and issues S_t = Q_t K^T
+//               (M=128, N=128, K=D as D/16 steps of 16) into TMEM.
+//   warp 10     (head_dim 96) issues O_t += P_t V (M=128, N=D, K=128 as 8
+//               steps, P read from TMEM, V as an MN-major operand).
+//   warp 11     idle: it completes the third warpgroup, whose registers
 //               (setmaxnreg) go to the softmax warpgroups (200 each).
-// TMEM columns: S_0 [0,128), S_1 [128,256), O_0 [256,352), O_1 [352,448) at
-// head_dim 96; the same kernel is instantiated for head_dim 128 (O_0
-// [256,384), O_1 [384,512), four 32-channel chunks per tile, 2-stage rings).
-// Every mbarrier wait is bounded (timeout + CTA abort flag); a timeout sets the
-// device status word instead of hanging or trapping.
+// Head_dim 96 (TMEM: S_0 [0,128), S_1 [128,256), O_0 [256,352), O_1
+// [352,448), P [448,512)): P goes to its own 64-column buffer, which the two
+// tiles take in turn, so S_t is released as soon as the softmax has read it
+// and QK_t(j+1) runs during the exponentials of block j; QK and PV have
+// separate issuing threads (warps 9 and 10), since they touch disjoint TMEM
+// and one thread's barrier latency would otherwise hold up the other's MMAs.
+// Head_dim 128 (O_0 [256,384), O_1 [384,512): no columns left): P_t is
+// written over S_t, 16 columns at a time, and warp 9 issues both MMAs in the
+// order PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1), so each softmax group waits
+// only on its own tile's chain; four 32-channel chunks per tile, 2-stage
+// rings.  Every mbarrier wait is bounded (timeout + CTA abort flag); a timeout
+// sets the device status word instead of hanging or trapping.
 #include <cuda_bf16.h>
 
 #include "h3a_internal.h"
@@ -48,11 +52,11 @@ namespace h3a {
 namespace {
 
 constexpr int kSoftmaxWarps = 8;                   // 2 warpgroups: one per query tile
-constexpr int kProducerWarp = 8, kMmaWarp = 9;
-constexpr int kThreads = 32 * (kSoftmaxWarps + 4);  // 384: warps 10-11 idle (a full third warpgroup)
+constexpr int kProducerWarp = 8, kMmaWarp = 9, kPvWarp = 10;
+constexpr int kThreads = 32 * (kSoftmaxWarps + 4);  // 384: a full third warpgroup (warp 11 idle)
 // Register split (setmaxnreg, per warpgroup): the launch gives every thread
 // 168 registers (65,536 / 384 rounded down to 8); the third warpgroup
-// (producer, MMA issuer, two idle warps) drops to 80 and the two softmax
+// (producer, MMA issuers, an idle warp) drops to 80 and the two softmax
 // warpgroups rise to 200, so a softmax thread holds its 128-value row without
 // spilling.  The new total must fit in what the block was launched with.
 constexpr uint32_t kRegsLaunch = (65536 / kThreads) / 8 * 8;
@@ -76,6 +80,13 @@ struct Geo {
     static constexpr int kStages = D == 96 ? 3 : 2;
     static constexpr int kKSteps = D / 16;  // QK^T k-steps of 16
     __host__ __device__ static constexpr uint32_t col_o(int t) { return 256u + (t ? D : 0); }
+    // At D = 96 the 64 columns after O_1 hold one bf16 P buffer that both
+    // tiles take in turn, so S_t is free as soon as its softmax has read it
+    // and QK_t(j+1) runs during the exponentials of block j.  At D = 128 no
+    // columns are left: P_t is written over S_t and QK_t(j+1) follows PV_t(j).
+    static constexpr bool kSepP = D == 96;
+    static constexpr uint32_t kColP = 256u + 2 * D;
+    static_assert(!kSepP || kColP + 64 <= kTmemCols, "P buffer inside the allocation");
 };
 
 template <int D>
@@ -89,7 +100,9 @@ struct AttnSmem {
     uint64_t k_full[kStages], k_empty[kStages];
     uint64_t v_full[kStages], v_empty[kStages];
     uint64_t s_full[2], p_full[2], o_done[2];
-    uint64_t mma_drain;
+    uint64_t s_read[2];   // separate-P scheme: S_t has been read into registers
+    uint64_t pv_done[2];  // separate-P scheme: PV_t(j) has completed (P buffer free)
+    uint64_t mma_drain, pv_drain;
     uint32_t tmem_base;
     int abort_flag;
     int never;  // stays 0: abort flag for waits that must ignore an abort
@@ -266,8 +279,8 @@ __device__ __forceinline__ bool issue_pv(AttnSmem<D>& sm, const AttnArgs& a, Mma
     tc_fence_after_sync();
     constexpr uint32_t idesc = idesc_bf16_f32(128, D, 0, 1);
     const uint64_t dv = st.dv + stage * stage_step<D>();
-    const uint32_t d = tmem + Geo<D>::col_o(t), pa = tmem + col_s(t);
-    // P_t: keys 2c and 2c+1 packed in S column c
+    const uint32_t d = tmem + Geo<D>::col_o(t), pa = tmem + (Geo<D>::kSepP ? Geo<D>::kColP : col_s(t));
+    // P_t: keys 2c and 2c+1 packed in column c of the P buffer (or of S_t)
     mma_ts(d, pa, dv, idesc, first ? 0u : 1u);
 #pragma unroll
     for (int s = 1; s < 8; ++s) mma_ts(d, pa + 8 * s, dv + mnmajor_step(s), idesc, 1u);
@@ -275,6 +288,72 @@ __device__ __forceinline__ bool issue_pv(AttnSmem<D>& sm, const AttnArgs& a, Mma
     return true;
 }
 
+// Separate-P scheme: two issuing threads.  QK^T and PV touch disjoint TMEM
+// (S_t, versus the P buffer and O_t) and their hand-offs are separate
+// barriers, so the QK issuer (warp 9) and the PV issuer (warp 10) run
+// independently and neither's barrier latency holds up the other's MMAs.
+// QK_t(j+1) may be issued as soon as the softmax has read S_t(j) (s_read);
+// PV_t(j) as soon as P_t(j) is in the P buffer (p_full).
+template <int D>
+__device__ void qk_issuer(AttnSmem<D>& sm, const AttnArgs& a, uint32_t tmem, bool has1, const int32_t* l0,
+                          const int32_t* l1, volatile int* abort_flag) {
+    const int ntiles = has1 ? 2 : 1;
+    MmaState st;
+    st.dq[0] = kmajor_base(sm.q[0]);
+    st.dq[1] = kmajor_base(sm.q[1]);
+    st.dk = kmajor_base(sm.k[0]);
+    bool ok = true;
+    for (int t = 0; t < ntiles && ok; ++t) ok = mbar_wait(&sm.q_full[t], 0u, abort_flag, a.timeout_ns);
+    KvPlan p = kv_plan(l0, l1, has1, 0);
+    for (int t = 0; t < ntiles && ok; ++t) ok = issue_qk<D>(sm, a, st, tmem, t, p, abort_flag);
+    for (int j = 0; j + 1 < a.n_iter && ok; ++j) {
+        p = kv_plan(l0, l1, has1, j + 1);
+        for (int t = 0; t < ntiles && ok; ++t) {
+            if (!mbar_wait(&sm.s_read[t], static_cast<uint32_t>(j & 1), abort_flag, a.timeout_ns)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after_sync();
+            ok = issue_qk<D>(sm, a, st, tmem, t, p, abort_flag);
+        }
+    }
+    if (!ok) raise_timeout(a, abort_flag);
+    // Drain: every MMA this thread issued must have completed before TMEM is released.
+    tc_commit(&sm.mma_drain);
+    mbar_wait(&sm.mma_drain, 0u, &sm.never, a.timeout_ns);
+}
+
+template <int D>
+__device__ void pv_issuer(AttnSmem<D>& sm, const AttnArgs& a, uint32_t tmem, bool has1, const int32_t* l0,
+                          const int32_t* l1, volatile int* abort_flag) {
+    const int ntiles = has1 ? 2 : 1;
+    MmaState st;
+    st.dv = mnmajor_base(sm.v[0]);
+    bool ok = true;
+    for (int j = 0; j < a.n_iter && ok; ++j) {
+        const KvPlan p = kv_plan(l0, l1, has1, j);
+        for (int t = 0; t < ntiles && ok; ++t) {
+            if (!mbar_wait(&sm.p_full[t], static_cast<uint32_t>(j & 1), abort_flag, a.timeout_ns)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after_sync();
+            if (!issue_pv<D>(sm, a, st, tmem, t, p, j == 0, abort_flag)) {
+                ok = false;
+                break;
+            }
+            tc_commit(&sm.pv_done[t]);
+            if (j + 1 == a.n_iter) tc_commit(&sm.o_done[t]);
+        }
+    }
+    if (!ok) raise_timeout(a, abort_flag);
+    tc_commit(&sm.pv_drain);
+    mbar_wait(&sm.pv_drain, 0u, &sm.never, a.timeout_ns);
+}
+
+// P-over-S scheme: one issuing thread, PV_t(j) then QK_t(j+1) per tile (the
+// QK overwrites the S/P columns the PV reads; MMAs from one thread complete
+// in issue order).
 template <int D>
 __device__ void mma_issuer(AttnSmem<D>& sm, const AttnArgs& a, uint32_t tmem, bool has1, const int32_t* l0,
                            const int32_t* l1, volatile int* abort_flag) {
@@ -341,14 +420,32 @@ __device__ __noinline__ void rescale_o(uint32_t tO, float alpha) {
 
 // Softmax of query tile t: thread r owns row r (TMEM lane r), all 128 keys.
 template <int D>
-__device__ void softmax_group(AttnSmem<D>& sm, const AttnArgs& a, uint32_t tmem, int t, int b, int h, int qb,
-                              const int32_t* list, volatile int* abort_flag) {
+__device__ void softmax_group(AttnSmem<D>& sm, const AttnArgs& a, uint32_t tmem, int t, bool has1, int b, int h,
+                              int qb, const int32_t* list, volatile int* abort_flag) {
+    constexpr bool kSep = Geo<D>::kSepP;
     const int lane = threadIdx.x & 31;
     const int quarter = (threadIdx.x >> 5) & 3;  // TMEM lanes [32*quarter, 32*quarter + 32)
     const int row = quarter * 32 + lane;
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t tS = tmem + lane_addr + col_s(t);
     const uint32_t tO = tmem + lane_addr + Geo<D>::col_o(t);
+    const uint32_t tP = tmem + lane_addr + Geo<D>::kColP;
+    // Separate-P scheme: before this tile writes the shared P buffer at step j,
+    // the PV that last read it must have completed -- the other tile's PV of
+    // step j-1 (tile 0) or of step j (tile 1), or this tile's own PV of step
+    // j-1 when the CTA has one tile.  That PV was issued after PV_t(j-1), so
+    // its completion also leaves O_t stable for a rescale.  The wait names a
+    // phase at most one ahead of the barrier's last completed one (the next
+    // phase needs this tile's own P), so a parity wait is exact.
+    auto wait_p_buffer = [&](int j) -> bool {
+        const int u = has1 ? 1 - t : 0;
+        const int ph = (has1 && t == 1) ? j : j - 1;
+        if (ph < 0) return true;
+        const bool r = __all_sync(0xffffffffu, mbar_wait(&sm.pv_done[u], static_cast<uint32_t>(ph & 1), abort_flag,
+                                                         a.timeout_ns));
+        if (r) tc_fence_after_sync();
+        return r;
+    };
     const float c = a.scale_log2;
     float m_used = -INFINITY;  // row reference max of scaled logits (log2 units)
     float l = 0.f;             // running row sum of P
@@ -363,14 +460,19 @@ __device__ void softmax_group(AttnSmem<D>& sm, const AttnArgs& a, uint32_t tmem,
         const int kv = list ? __ldg(list + j) : j;
         const int valid = (kv == a.nblk - 1) ? a.N - kv * 128 : 128;
         // the whole row of S in registers: one wait, the true block max before
-        // any exponential, P packed in place over the same registers and
-        // stored in 16-column chunks as they complete (over S columns already
-        // read), so little store traffic is left to wait for at the end
+        // any exponential, P packed in place over the same registers
         uint32_t x[128];
 #pragma unroll
         for (int q = 0; q < 4; ++q) tmem_ld_x32(tS + 32u * q, slice32(x + 32 * q));
 #pragma unroll
         for (int q = 0; q < 4; ++q) tmem_wait_ld_x32(slice32(x + 32 * q));
+        if constexpr (kSep) {
+            // S_t is in registers: release it for QK_t(j+1)
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.s_read[t]);
+        }
+        bool p_free = false;  // separate-P scheme: the P buffer wait is done
         if (valid < 128) {
 #pragma unroll
             for (int i = 0; i < 128; ++i)
@@ -386,7 +488,15 @@ __device__ void softmax_group(AttnSmem<D>& sm, const AttnArgs& a, uint32_t tmem,
         } else {
             const bool need = mx - m_used > 8.0f;
             if (__any_sync(0xffffffffu, need)) {
-                // rare: O_t is stable here (the commit behind s_full covers PV_t(j-1))
+                // rare: O_t must be stable -- with P over S the commit behind
+                // s_full covers PV_t(j-1); with a separate P buffer, its wait does
+                if constexpr (kSep) {
+                    if (!wait_p_buffer(j)) {
+                        ok = false;
+                        break;
+                    }
+                    p_free = true;
+                }
                 float alpha = 1.0f;
                 if (need) {
                     alpha = ex2_approx(m_used - mx);
@@ -405,7 +515,18 @@ __device__ void softmax_group(AttnSmem<D>& sm, const AttnArgs& a, uint32_t tmem,
             const float p0 = ex2_approx(a0), p1 = ex2_approx(a1);
             acc[i & 1] = f2_add(acc[i & 1], f2(p0, p1));
             x[i] = pack_bf16x2(p0, p1);  // i < 2i: the S values read here are never needed again
-            if ((i & 15) == 15) tmem_st_x16(tS + (i - 15), slice16(x + (i - 15)));
+            // P over S: each 16-column chunk is stored as soon as it is
+            // complete (over S columns already read)
+            if constexpr (!kSep)
+                if ((i & 15) == 15) tmem_st_x16(tS + (i - 15), slice16(x + (i - 15)));
+        }
+        if constexpr (kSep) {
+            if (!p_free && !wait_p_buffer(j)) {
+                ok = false;
+                break;
+            }
+            tmem_st_x32(tP, slice32(x));
+            tmem_st_x32(tP + 32u, slice32(x + 32));
         }
         float s0, s1, s2, s3;
         f2_split(acc[0], s0, s1);
@@ -471,6 +592,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&sm.s_full[t], 1);
             mbar_init(&sm.p_full[t], 4);  // one arrival per softmax warp of the tile
             mbar_init(&sm.o_done[t], 1);
+            mbar_init(&sm.s_read[t], 4);  // one arrival per softmax warp of the tile
+            mbar_init(&sm.pv_done[t], 1);
         }
         for (int s = 0; s < Geo<D>::kStages; ++s) {
             mbar_init(&sm.k_full[s], 1);
@@ -479,6 +602,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&sm.v_empty[s], 1);
         }
         mbar_init(&sm.mma_drain, 1);
+        mbar_init(&sm.pv_drain, 1);
         sm.abort_flag = 0;
         sm.never = 0;
         fence_barrier_init();
@@ -496,13 +620,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp < kSoftmaxWarps) {
         asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
         const int t = warp >> 2;  // softmax warpgroup = query tile
-        if (t == 0 || has1) softmax_group<D>(sm, a, tmem, t, b, h, qb0 + t, t ? l1 : l0, abort_flag);
+        if (t == 0 || has1) softmax_group<D>(sm, a, tmem, t, has1, b, h, qb0 + t, t ? l1 : l0, abort_flag);
     } else {
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsOther));
         if (warp == kProducerWarp) {
             if ((threadIdx.x & 31) == 0) producer<D>(sm, a, &tq, &tk, &tv, b, h, qb0, has1, l0, l1, abort_flag);
         } else if (warp == kMmaWarp) {
-            if ((threadIdx.x & 31) == 0) mma_issuer<D>(sm, a, tmem, has1, l0, l1, abort_flag);
+            if ((threadIdx.x & 31) == 0) {
+                if constexpr (Geo<D>::kSepP)
+                    qk_issuer<D>(sm, a, tmem, has1, l0, l1, abort_flag);
+                else
+                    mma_issuer<D>(sm, a, tmem, has1, l0, l1, abort_flag);
+            }
+        } else if (warp == kPvWarp) {
+            if constexpr (Geo<D>::kSepP)
+                if ((threadIdx.x & 31) == 0) pv_issuer<D>(sm, a, tmem, has1, l0, l1, abort_flag);
         }
     }
     tc_fence_before_sync();
