@@ -7,7 +7,10 @@ One step = the whole hot path over one batch of the 5 s 1344x768 clip latent
     ->  dense attention
 The headline value is attention TFLOP/s over the whole step (algorithmic
 FLOPs of both attention passes / step time).  Per-kernel times come from CUDA
-events on the launching stream inside the timed region.
+events on the launching stream inside the timed region.  Beside the headline,
+outside the timed step, the same four launches run on the 10 s clip
+(61x48x84 = 245,952 tokens, sparsity 0.80) and are reported under
+kernels.video10s_untimed_step (--no-video10s skips them).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 
@@ -301,6 +304,10 @@ def run_gpu(args, rank, world, local):
         torch.cuda.synchronize()
         kern_ms["prologue_fullnorm"] = allreduce_max(fe[0].elapsed_time(fe[1]), world)
     dit = time_dit_ops(h3a, synth, q, k, B, N, heads * w.head_dim, stream, world, rank)
+    pk, pk_src = peaks()
+    video10s = None
+    if args.video10s and not wide:
+        video10s = time_video10s(h3a, synth, stream, world, rank, pk)
     if wide:
         kern_ms["prologue"] = kern_ms["prologue_pool"] = 0.0
         kern_ms["router"] = kern_ms["router_scores"]
@@ -395,7 +402,6 @@ def run_gpu(args, rank, world, local):
     if rank != 0:
         return None
 
-    pk, pk_src = peaks()
     dense_tflops = flops_dense / (kern_ms["attention_dense"] * 1e-3) / 1e12
     sparse_tflops = flops_sparse / (kern_ms["attention_sparse"] * 1e-3) / 1e12
     D = w.head_dim
@@ -464,7 +470,7 @@ def run_gpu(args, rank, world, local):
                                                 (kern_ms["attention_sparse"] + route_cost), 3),
         } | {name: dict(ent, frac_hbm=round(ent["GB/s"] / pk["hbm_gbs"], 4),
                         traffic=traffic.get(ent.pop("traffic_key"), {}).get("bytes_per_launch"))
-             for name, ent in dit.items()},
+             for name, ent in dit.items()} | ({"video10s_untimed_step": video10s} if video10s else {}),
         "gpu_launches": args.steps * 4,
         "clocks": clocks,
         "e2e": e2e,
@@ -472,6 +478,72 @@ def run_gpu(args, rank, world, local):
     if args.cpu_baseline and world == 1:
         line["cpu_baseline"] = cpu_baseline(d, w, args.cpu_rows)
     return line
+
+
+def time_video10s(h3a, synth, stream, world, rank, pk, reps=2):
+    """The 10 s clip (61x48x84 = 245,952 tokens, 56 heads x 96), outside the
+    timed step: the same four launches as a step -- prologue with pooling,
+    router scores/top-k at sparsity 0.80, sparse attention, dense attention --
+    one untimed pass, then `reps` timed with CUDA events on the launching
+    stream.  Returns the per-kernel times, dense and sparse TFLOP/s, their
+    fractions of the measured bf16 peaks and the sparse/dense wall-clock ratio
+    with routing charged to the sparse path."""
+    name, sparsity = "video10s", 0.80
+    w = synth.WORKLOADS[name]
+    d = synth.draw_workload(name, seed=rank)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    q, k, v = (d[n].to(dev) for n in "qkv")
+    gq, gk = d["gamma_q"].to(dev), d["gamma_k"].to(dev)
+    del d
+    qn, kn = torch.empty_like(q), torch.empty_like(k)
+    o_dense, o_sparse = torch.empty_like(q), torch.empty_like(q)
+    nblk = (w.N + 127) // 128
+    kk = h3a.route_k(nblk, sparsity)
+    blocks = torch.empty((w.B, w.heads, nblk, kk), dtype=torch.int32, device=dev)
+    ws = torch.empty(h3a.route_workspace_size(q), dtype=torch.uint8, device=dev)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(reps + 1)]
+    for i in range(reps + 1):
+        ev = evs[i]
+        ev[0].record(stream)
+        h3a.qk_norm_rope_pool(q, k, gq, gk, w.grid, workspace=ws, out=(qn, kn))
+        ev[1].record(stream)
+        h3a.route_pooled(qn, sparsity, ws, out=blocks)
+        ev[2].record(stream)
+        h3a.attention(qn, kn, v, blocks, out=o_sparse)
+        ev[3].record(stream)
+        h3a.attention(qn, kn, v, None, out=o_dense)
+        ev[4].record(stream)
+    torch.cuda.synchronize()
+    if h3a.last_device_error() != 0:
+        raise RuntimeError("device-side timeout in the 245,952-token pass")
+    ms = [allreduce_max(float(np.mean([evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(1, reps + 1)])), world)
+          for j in range(4)]
+    flops_dense = attention_flops(w.N, w.heads, w.B)
+    flops_sparse = attention_flops(w.N, w.heads, w.B, blocks=blocks.cpu().numpy())
+    pro_bytes = prologue_bytes(w.N, w.heads, w.B) + pooled_bytes(w.N, w.heads, w.B)
+    dense_t = flops_dense / (ms[3] * 1e-3) / 1e12
+    sparse_t = flops_sparse / (ms[2] * 1e-3) / 1e12
+    del q, k, v, qn, kn, o_dense, o_sparse, blocks, ws
+    torch.cuda.empty_cache()
+    return {
+        "workload": f"{name}: B=1, 56 heads x 96, grid 61x48x84 = {w.N:,} tokens; prologue with block pooling + "
+                    f"router scores/top-k (sparsity {sparsity}, k={kk}/{nblk}) + sparse + dense attention; "
+                    f"{reps} timed passes after one untimed",
+        "prologue_pool_ms": round(ms[0], 4),
+        "prologue_pool_GB/s": round(pro_bytes / (ms[0] * 1e-3) / 1e9, 1),
+        "router_scores_ms": round(ms[1], 4),
+        "attention_sparse_ms": round(ms[2], 3),
+        "attention_dense_ms": round(ms[3], 3),
+        "dense_TFLOP/s": round(dense_t, 2),
+        "dense_frac_sustained": round(dense_t / pk["bf16_tflops_sustained"], 4),
+        "dense_frac_burst": round(dense_t / pk["bf16_tflops"], 4),
+        "sparse_TFLOP/s": round(sparse_t, 2),
+        "sparse_frac_sustained": round(sparse_t / pk["bf16_tflops_sustained"], 4),
+        "sparse_effective_dense_equiv_TFLOP/s": round(flops_dense / (ms[2] * 1e-3) / 1e12, 2),
+        "algorithmic_flops_dense": flops_dense,
+        "algorithmic_flops_sparse": flops_sparse,
+        "sparse_speedup_incl_router": round(ms[3] / (ms[2] + ms[1]), 3),
+    }
 
 
 def time_dit_ops(h3a, synth, q, k, B, N, width, stream, world, rank, reps=10):
@@ -624,6 +696,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--cpu-rows", type=int, default=4096, help="query rows of the CPU-baseline sample")
     ap.add_argument("--ref-rows", type=int, default=128, help="query rows per reference-arm step")
+    ap.add_argument("--no-video10s", dest="video10s", action="store_false",
+                    help="skip the 245,952-token pass reported beside the headline")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

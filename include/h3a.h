@@ -16,15 +16,20 @@
  *     channels).  block must be 128.
  *   - All pointers are DEVICE pointers owned by the caller, 16-byte aligned;
  *     strides are multiples of 8 elements (16 bytes).  The library never
- *     allocates or frees device memory; the router's scratch is a caller
- *     workspace sized by h3a_route_workspace_size.
+ *     allocates or frees device memory per call; the router's scratch is a
+ *     caller workspace sized by h3a_route_workspace_size.  Its only device
+ *     state is static: the status word below and the fixed scratch array of
+ *     h3a_route_noalloc, both resident on every GPU that loads the library.
  *   - Calls are asynchronous on the caller's stream.  A status other than
  *     H3A_OK means nothing was launched, except H3A_ERR_CUDA, returned when a
  *     launch itself failed.  Device-side failures (a bounded pipeline wait that
  *     expired) are latched in a per-device status word and reported by
  *     h3a_last_device_error.
- *   - Thread safety: calls may be issued from several host threads; a call
- *     touches only its arguments and read-only per-process state.
+ *   - Thread safety: calls may be issued from several host threads.  A call
+ *     writes only its arguments, except for two pieces of shared device state:
+ *     kernels OR timeouts into the per-device status word (taken atomically by
+ *     h3a_last_device_error), and h3a_route_noalloc works in one scratch array
+ *     per device, so its calls race when they overlap on the GPU.
  */
 #ifndef H3A_H_
 #define H3A_H_
@@ -218,8 +223,10 @@ h3a_status h3a_residual_diff(const void* cur, const void* prev, int64_t n, doubl
                              void* workspace, size_t ws_bytes, double* rel_out, int32_t* reuse_out,
                              h3a_stream_t stream);
 
-/* Capacity of the scratch built into h3a_route_noalloc: 64 MiB, enough for
- * B * heads * ceil(N / 128) <= 87,381 (e.g. 56 heads of a 124,992-token clip). */
+/* Capacity of the scratch built into h3a_route_noalloc: 64 MiB.  The router
+ * keeps two fp32 block means of head_dim values per (batch, head, block), so it
+ * holds B * heads * ceil(N / 128) <= 64 MiB / (8 * head_dim) blocks: 87,381 at
+ * head_dim 96 (e.g. 56 heads of a 124,992-token clip), 65,536 at 128. */
 #define H3A_ROUTE_NOALLOC_MAX_BYTES ((size_t)64 << 20)
 
 /* h3a_route for callers that cannot allocate device memory (no counterpart on
@@ -269,9 +276,15 @@ const char* h3a_status_string(h3a_status s);
 /* Text of the last CUDA error seen by the calling host thread ("" if none). */
 const char* h3a_last_cuda_error_string(void);
 
-/* Synchronises `stream`, then reads and clears the current device's status
- * word: H3A_OK, or H3A_ERR_TIMEOUT if a bounded device wait expired since the
- * last read.  H3A_ERR_CUDA if the synchronisation itself failed. */
+/* Takes the current device's status word: after everything already queued
+ * on `stream`, one atomic exchange reads the word and clears it, then the call
+ * synchronises `stream` and returns H3A_OK, or H3A_ERR_TIMEOUT if a bounded
+ * device wait expired since the word was last taken.  The word is shared by
+ * every stream of the device: a timeout raised by a kernel on another stream is
+ * reported to exactly one caller -- this one if that kernel had already raised
+ * it, else a later one; it is never lost, and never reported twice.  Readers
+ * in one process are serialised.  H3A_ERR_CUDA if the launch, the copy or the
+ * synchronisation failed. */
 h3a_status h3a_last_device_error(h3a_stream_t stream);
 
 /* Self-check of the bounded-wait path (no counterpart on the pages): launches
@@ -292,14 +305,12 @@ h3a_status h3a_selftest_wait_timeout(uint32_t limit_us, h3a_stream_t stream);
 h3a_status h3a_selftest_mma(const void* a, const void* b, float* s_out, float* r_out,
                             h3a_stream_t stream);
 
-/* Self-check of the exponentials of the attention softmax (no counterpart on
- * the pages): y[i] = 2^x[i] for n device floats, computed by the same device
- * code the softmax uses -- the FMA-pipe polynomial (use_poly != 0: Cody-Waite
- * split x = n + f with f in [-1/2, 1/2], degree-3 minimax polynomial for 2^f,
- * max relative error 7.5e-5 for x >= -125; x below -126 is clamped there and
- * yields at most 2^-125) or ex2.approx (use_poly == 0).  Asynchronous on
- * `stream`.  INVALID_ARG for n < 0 or null / misaligned pointers. */
-h3a_status h3a_selftest_exp2(const float* x, float* y, int32_t n, int32_t use_poly, h3a_stream_t stream);
+/* Self-check of the exponential of the attention softmax (no counterpart on
+ * the pages): y[i] = 2^x[i] for n device floats, by the instruction the
+ * softmax evaluates every exponential with (ex2.approx.ftz.f32, in the log2
+ * domain).  Asynchronous on `stream`.  INVALID_ARG for n < 0 or null /
+ * misaligned pointers. */
+h3a_status h3a_selftest_exp2(const float* x, float* y, int32_t n, h3a_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -1,6 +1,7 @@
 // C-ABI front end of libh3a: argument validation, tensor-map encoding and
 // launches on the caller's stream.  Nothing here allocates device memory; the
-// only device state is the per-device status word below.
+// only device state is the per-device status word below (and the copy of it
+// that the last read took).
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -15,6 +16,13 @@
 
 // Sticky per-device status word: kernels OR error bits into it.
 __device__ int g_h3a_status_word;
+// What the last read of the status word took out of it.
+__device__ int g_h3a_status_taken;
+
+// Reads and clears the status word in one atomic step, so that an error a
+// kernel on another stream ORs in at the same moment is either taken by this
+// read or left for the next one -- never lost.
+__global__ void status_take_kernel() { g_h3a_status_taken = atomicExch(&g_h3a_status_word, 0); }
 
 namespace h3a {
 namespace {
@@ -31,6 +39,8 @@ h3a_status cuda_fail(cudaError_t e) {
 
 // Device address of g_h3a_status_word, resolved once per device.
 std::mutex g_status_mu;
+// Serialises readers of g_h3a_status_taken (one per process at a time).
+std::mutex g_take_mu;
 int* g_status_ptr[kMaxDevices] = {};
 
 h3a_status status_word(int** out) {
@@ -343,12 +353,15 @@ h3a_status h3a_last_device_error(h3a_stream_t stream) {
     int* status = nullptr;
     h3a_status rc = status_word(&status);
     if (rc != H3A_OK) return rc;
-    cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
-    if (e != cudaSuccess) return cuda_fail(e);
+    const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    std::lock_guard<std::mutex> lock(g_take_mu);
+    // after everything already queued on `stream`: take the word, then copy it out
+    status_take_kernel<<<1, 1, 0, st>>>();
+    cudaError_t e = cudaGetLastError();
     int word = 0;
-    const int zero = 0;
-    e = cudaMemcpyFromSymbol(&word, g_h3a_status_word, sizeof(int));
-    if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_h3a_status_word, &zero, sizeof(int));
+    if (e == cudaSuccess) e = cudaMemcpyFromSymbolAsync(&word, g_h3a_status_taken, sizeof(int), 0,
+                                                        cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
     if (e != cudaSuccess) return cuda_fail(e);
     return (word & kDevTimeout) ? H3A_ERR_TIMEOUT : H3A_OK;
 }
@@ -380,10 +393,10 @@ h3a_status h3a_selftest_mma(const void* a, const void* b, float* s_out, float* r
     return e == cudaSuccess ? H3A_OK : cuda_fail(e);
 }
 
-h3a_status h3a_selftest_exp2(const float* x, float* y, int32_t n, int32_t use_poly, h3a_stream_t stream) {
+h3a_status h3a_selftest_exp2(const float* x, float* y, int32_t n, h3a_stream_t stream) {
     if (n < 0 || (n > 0 && (!x || !y))) return H3A_ERR_INVALID_ARG;
     if ((reinterpret_cast<uintptr_t>(x) & 3u) || (reinterpret_cast<uintptr_t>(y) & 3u)) return H3A_ERR_INVALID_ARG;
-    cudaError_t e = launch_selftest_exp2(x, y, n, use_poly ? 1 : 0, reinterpret_cast<cudaStream_t>(stream));
+    cudaError_t e = launch_selftest_exp2(x, y, n, reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? H3A_OK : cuda_fail(e);
 }
 

@@ -65,7 +65,7 @@ cudaError_t launch_residual_diff(const void* cur, const void* prev, int64_t n, d
 
 // Self-checks (selftest.cu).
 cudaError_t launch_selftest_wait(uint64_t limit_ns, int* status, cudaStream_t st);
-cudaError_t launch_selftest_exp2(const float* x, float* y, int n, int poly, cudaStream_t st);
+cudaError_t launch_selftest_exp2(const float* x, float* y, int n, cudaStream_t st);
 cudaError_t launch_selftest_mma(const CUtensorMap& ta, const CUtensorMap& tb, float* s_out, float* r_out,
                                 int* status, uint64_t timeout_ns, cudaStream_t st);
 

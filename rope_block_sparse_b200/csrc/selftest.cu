@@ -7,8 +7,8 @@
 //                        tiles, S = A B^T into TMEM (K-major operands), bf16(S)
 //                        written back to TMEM, R = bf16(S) B with B read as an
 //                        MN-major operand and A taken from TMEM.
-//   exp2_selftest_kernel evaluates the softmax's FMA-pipe exp2 polynomial (or
-//                        ex2.approx) element-wise, for checking it against 2^x.
+//   exp2_selftest_kernel evaluates the softmax's exponential (ex2.approx)
+//                        element-wise, for checking it against 2^x.
 #include "fastmath.cuh"
 #include "h3a_internal.h"
 #include "sm100.cuh"
@@ -139,27 +139,16 @@ __global__ void __launch_bounds__(128, 1)
     }
 }
 
-__global__ void exp2_selftest_kernel(const float* x, float* y, int n, int poly) {
-    const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
-    if (i >= n) return;
-    const float x0 = x[i], x1 = (i + 1 < n) ? x[i + 1] : 0.f;
-    float y0, y1;
-    if (poly) {
-        f2_split(exp2_poly_pair(f2(x0, x1)), y0, y1);
-    } else {
-        y0 = ex2_approx(x0);
-        y1 = ex2_approx(x1);
-    }
-    y[i] = y0;
-    if (i + 1 < n) y[i + 1] = y1;
+__global__ void exp2_selftest_kernel(const float* x, float* y, int n) {
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i < n) y[i] = ex2_approx(x[i]);
 }
 
 }  // namespace
 
-cudaError_t launch_selftest_exp2(const float* x, float* y, int n, int poly, cudaStream_t st) {
+cudaError_t launch_selftest_exp2(const float* x, float* y, int n, cudaStream_t st) {
     if (n <= 0) return cudaSuccess;
-    const int pairs = (n + 1) / 2;
-    exp2_selftest_kernel<<<(pairs + 255) / 256, 256, 0, st>>>(x, y, n, poly);
+    exp2_selftest_kernel<<<(n + 255) / 256, 256, 0, st>>>(x, y, n);
     return cudaGetLastError();
 }
 

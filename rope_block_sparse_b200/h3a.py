@@ -86,7 +86,7 @@ def load() -> ctypes.CDLL:
     lib.h3a_selftest_wait_timeout.restype = st
     lib.h3a_selftest_mma.argtypes = [P, P, P, P, P]
     lib.h3a_selftest_mma.restype = st
-    lib.h3a_selftest_exp2.argtypes = [P, P, i32, i32, P]
+    lib.h3a_selftest_exp2.argtypes = [P, P, i32, P]
     lib.h3a_selftest_exp2.restype = st
     lib.h3a_route_noalloc.argtypes = [P, P, ctypes.POINTER(QkvDesc), f64, i32, P, ctypes.POINTER(ctypes.c_int64), P]
     lib.h3a_route_noalloc.restype = st
@@ -399,13 +399,13 @@ def selftest_mma(a: torch.Tensor, b: torch.Tensor):
     return s, r
 
 
-def selftest_exp2(x: torch.Tensor, use_poly: bool = True) -> torch.Tensor:
-    """2^x by the softmax's exponential (FMA-pipe polynomial, or ex2.approx): fp32 CUDA tensor in and out."""
+def selftest_exp2(x: torch.Tensor) -> torch.Tensor:
+    """2^x by the softmax's exponential (ex2.approx): fp32 CUDA tensor in and out."""
     lib = load()
     if not x.is_cuda or x.dtype != torch.float32 or not x.is_contiguous():
         raise ValueError("x must be a contiguous fp32 CUDA tensor")
     y = torch.empty_like(x)
-    _check("h3a_selftest_exp2", lib.h3a_selftest_exp2(_ptr(x), _ptr(y), x.numel(), int(use_poly), _stream_handle()))
+    _check("h3a_selftest_exp2", lib.h3a_selftest_exp2(_ptr(x), _ptr(y), x.numel(), _stream_handle()))
     return y
 
 
