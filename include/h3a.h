@@ -113,9 +113,11 @@ h3a_status h3a_qk_fullnorm_rope(const void* q, const void* k, const h3a_qkv_desc
  * Host only; no device work. */
 double h3a_step_sparsity(int32_t step, int32_t first_sparse_step, double sparsity);
 
-/* Bytes of device workspace h3a_route needs: two fp32 [B, heads, nblk,
- * head_dim] pooled tensors, nblk = ceil(N / block), head_dim 96 or 128.
- * Returns INVALID_ARG/UNSUPPORTED for bad descriptors. */
+/* Bytes of device workspace h3a_route needs for the fp32 block means,
+ * nblk = ceil(N / block), head_dim 96 or 128: Q's as [B, heads, nblk,
+ * head_dim], then, from the next 256-byte boundary, K's channel-major as
+ * [B, heads, head_dim, nblk rounded up to 4], each part rounded up to 256
+ * bytes.  Returns INVALID_ARG/UNSUPPORTED for bad descriptors. */
 h3a_status h3a_route_workspace_size(const h3a_qkv_desc* d, int32_t block, size_t* bytes);
 
 /* Blockwise KV-block router.
@@ -146,8 +148,8 @@ h3a_status h3a_route(const void* q, const void* k, const h3a_qkv_desc* d, double
  * Writes q_out / k_out exactly as h3a_qk_norm_rope does, and into workspace
  * the fp32 means, over each 128-token block (the tail block over its real
  * length), of the rounded outputs: the same bytes h3a_route's pooling leaves
- * in its workspace (two fp32 [B, heads, nblk, 96] tensors, Q's first, at the
- * offsets h3a_route uses), bit for bit.
+ * in its workspace (the layout h3a_route_workspace_size describes), bit for
+ * bit.
  * workspace : device, at least h3a_route_workspace_size(d, 128) bytes,
  *             16-B aligned, owned by the caller; it must not overlap q, k,
  *             q_out or k_out.
@@ -224,9 +226,11 @@ h3a_status h3a_residual_diff(const void* cur, const void* prev, int64_t n, doubl
                              h3a_stream_t stream);
 
 /* Capacity of the scratch built into h3a_route_noalloc: 64 MiB.  The router
- * keeps two fp32 block means of head_dim values per (batch, head, block), so it
- * holds B * heads * ceil(N / 128) <= 64 MiB / (8 * head_dim) blocks: 87,381 at
- * head_dim 96 (e.g. 56 heads of a 124,992-token clip), 65,536 at 128. */
+ * keeps two fp32 block means of head_dim values per (batch, head, block) (the
+ * layout h3a_route_workspace_size gives), so it holds about
+ * B * heads * ceil(N / 128) <= 64 MiB / (8 * head_dim) blocks: some 87,000 at
+ * head_dim 96 (e.g. 56 heads of a 124,992-token clip), 65,000 at 128; a shape
+ * whose workspace size exceeds 64 MiB is refused. */
 #define H3A_ROUTE_NOALLOC_MAX_BYTES ((size_t)64 << 20)
 
 /* h3a_route for callers that cannot allocate device memory (no counterpart on

@@ -92,8 +92,14 @@ h3a_status check_desc(const h3a_qkv_desc* d, Shape* s, bool wide_ok = false) {
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-size_t pooled_bytes(const Shape& s, int nblk) {
+// Router workspace: the fp32 block means of Q, [B, heads, nblk, d], then those
+// of K stored channel-major, [B, heads, d, pooled_k_stride(nblk)], each half
+// starting on a 256-byte boundary.
+size_t pooled_q_bytes(const Shape& s, int nblk) {
     return align256(static_cast<size_t>(s.B) * s.heads * nblk * s.d * sizeof(float));
+}
+size_t pooled_k_bytes(const Shape& s, int nblk) {
+    return align256(static_cast<size_t>(s.B) * s.heads * s.d * pooled_k_stride(nblk) * sizeof(float));
 }
 
 }  // namespace
@@ -135,8 +141,9 @@ h3a_status route_setup(const Shape& s, double sparsity, int32_t block, const voi
     *nblk = (s.N + kBlock - 1) / kBlock;
     if (*nblk > route_max_blocks(s.d)) return H3A_ERR_UNSUPPORTED;
     if (static_cast<int64_t>(s.B) * s.heads > 65535) return H3A_ERR_UNSUPPORTED;
-    const size_t half = pooled_bytes(s, *nblk);
-    if (workspace == nullptr || !aligned16(workspace) || ws_bytes < 2 * half) return H3A_ERR_WORKSPACE;
+    const size_t half = pooled_q_bytes(s, *nblk);
+    if (workspace == nullptr || !aligned16(workspace) || ws_bytes < half + pooled_k_bytes(s, *nblk))
+        return H3A_ERR_WORKSPACE;
     *kk = h3a_route_k(*nblk, sparsity);
     *pq = static_cast<float*>(const_cast<void*>(workspace));
     *pk = reinterpret_cast<float*>(static_cast<char*>(const_cast<void*>(workspace)) + half);
@@ -222,7 +229,7 @@ h3a_status h3a_route_workspace_size(const h3a_qkv_desc* d, int32_t block, size_t
     if (bytes == nullptr) return H3A_ERR_INVALID_ARG;
     if (block != kBlock) return H3A_ERR_UNSUPPORTED;
     const int nblk = (s.N + kBlock - 1) / kBlock;
-    *bytes = 2 * pooled_bytes(s, nblk);
+    *bytes = pooled_q_bytes(s, nblk) + pooled_k_bytes(s, nblk);
     return H3A_OK;
 }
 
@@ -253,8 +260,9 @@ h3a_status h3a_qk_norm_rope_pool(const void* q, const void* k, const h3a_qkv_des
     if (rc != H3A_OK) return rc;
     const int nblk = (s.N + kBlock - 1) / kBlock;
     if (s.B > 65535 || (s.heads + 27) / 28 > 65535) return H3A_ERR_UNSUPPORTED;
-    const size_t half = pooled_bytes(s, nblk);
-    if (workspace == nullptr || !aligned16(workspace) || ws_bytes < 2 * half) return H3A_ERR_WORKSPACE;
+    const size_t half = pooled_q_bytes(s, nblk);
+    if (workspace == nullptr || !aligned16(workspace) || ws_bytes < half + pooled_k_bytes(s, nblk))
+        return H3A_ERR_WORKSPACE;
     float* pq = static_cast<float*>(workspace);
     float* pk = reinterpret_cast<float*>(static_cast<char*>(workspace) + half);
     cudaError_t e = launch_qk_norm_rope_pool(q, k, q_out, k_out, gamma_q, gamma_k, s, grid.H, grid.W, theta, eps, pq,

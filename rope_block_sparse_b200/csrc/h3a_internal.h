@@ -32,13 +32,18 @@ cudaError_t launch_qk_fullnorm_rope(const void* q, const void* k, void* q_out, v
                                     cudaStream_t st);
 
 // Prologue that also writes the fp32 means of its rounded outputs over
-// 128-token blocks into pool_q / pool_k ([B, heads, nblk, 96]) (prologue.cu).
+// 128-token blocks into pool_q / pool_k (the router's layouts, below) (prologue.cu).
 cudaError_t launch_qk_norm_rope_pool(const void* q, const void* k, void* q_out, void* k_out, const float* gamma_q,
                                      const float* gamma_k, const Shape& s, int H, int W, double theta, float eps,
                                      float* pool_q, float* pool_k, cudaStream_t st);
 
-// Router (router.cu): block means of q and k into pooled_q / pooled_k
-// ([B, heads, nblk, 96] fp32), then scores and top-k into idx.
+// The router's fp32 block means: Q's as [B, heads, nblk, d]; K's channel-major,
+// [B, heads, d, pooled_k_stride(nblk)] (one 16-byte-aligned row of key blocks
+// per channel, so that the score kernel reads consecutive key blocks).
+__host__ __device__ inline int pooled_k_stride(int nblk) { return (nblk + 3) & ~3; }
+
+// Router (router.cu): block means of q and k into pooled_q / pooled_k (the
+// layouts above), then scores and top-k into idx.
 cudaError_t launch_route(const void* q, const void* k, const Shape& s, int nblk, int kk, float* pooled_q,
                          float* pooled_k, int32_t* idx, cudaStream_t st);
 // Scores and top-k only, from block means already in pooled_q / pooled_k.

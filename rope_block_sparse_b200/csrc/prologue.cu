@@ -280,16 +280,18 @@ __global__ void __launch_bounds__(kPoolThreads, 2) qk_norm_rope_pool_kernel(cons
     }
     if (!active) return;
     const float inv_len = 1.0f / static_cast<float>(len);
-    const int64_t dst = ((static_cast<int64_t>(b) * a.heads + h) * a.nblk + blk) * kHeadDim + c0;
-    float4* dq = reinterpret_cast<float4*>(a.pool_q + dst);
-    float4* dk = reinterpret_cast<float4*>(a.pool_k + dst);
+    // Q's means row-major [B, heads, nblk, 96]; K's channel-major
+    // [B, heads, 96, stride], the router's layouts
+    const int64_t bh = static_cast<int64_t>(b) * a.heads + h;
+    float4* dq = reinterpret_cast<float4*>(a.pool_q + (bh * a.nblk + blk) * kHeadDim + c0);
 #pragma unroll
-    for (int u = 0; u < kChanPerLane / 4; ++u) {
+    for (int u = 0; u < kChanPerLane / 4; ++u)
         dq[u] = make_float4(accq[4 * u] * inv_len, accq[4 * u + 1] * inv_len, accq[4 * u + 2] * inv_len,
                             accq[4 * u + 3] * inv_len);
-        dk[u] = make_float4(acck[4 * u] * inv_len, acck[4 * u + 1] * inv_len, acck[4 * u + 2] * inv_len,
-                            acck[4 * u + 3] * inv_len);
-    }
+    const int kstride = pooled_k_stride(a.nblk);
+    float* dk = a.pool_k + (bh * kHeadDim + c0) * kstride + blk;
+#pragma unroll
+    for (int i = 0; i < kChanPerLane; ++i) dk[static_cast<int64_t>(i) * kstride] = acck[i] * inv_len;
 }
 
 // ---------------------------------------------------------------------------

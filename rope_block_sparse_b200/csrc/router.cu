@@ -7,10 +7,12 @@
 // Two kernels:
 //   block_pool_kernel   HBM-bound: one CTA per (batch, block, tensor) streams the
 //                       block's 128 token rows (all heads) once and writes fp32
-//                       means [B, heads, nblk, 96].
+//                       means: Q's [B, heads, nblk, D], K's channel-major
+//                       [B, heads, D, nblk rounded up to 4].
 //   score_topk_kernel   one CTA per (batch*head, 16 query blocks): fp32 scores of
 //                       its query blocks against every key block into shared
-//                       memory, then one warp per query block selects the top k
+//                       memory (8 x 4 register tiles over the channel-major K
+//                       means), then one warp per query block selects the top k
 //                       with a 4-pass 8-bit radix select over order-preserving
 //                       32-bit keys and emits the indices in ascending order.
 #include <cuda_bf16.h>
@@ -98,16 +100,24 @@ __global__ void __launch_bounds__(kPoolThreads) block_pool_kernel(const PoolArgs
             if (act[u]) acc8(acc[u], __ldg(reinterpret_cast<const uint4*>(x + off[u] + static_cast<int64_t>(n) * a.sn)));
     }
     const float inv_len = 1.0f / static_cast<float>(n1 - n0);
+    const int kstride = pooled_k_stride(a.nblk);
 #pragma unroll
     for (int u = 0; u < kVecPerThread; ++u) {
         if (!act[u]) continue;
         const int v = threadIdx.x + u * kPoolThreads;
         const int h = h_base + v / kVecPerHead, c = (v % kVecPerHead) * 8;
-        float* dst = a.out[which] + ((static_cast<int64_t>(b) * a.heads + h) * a.nblk + blk) * D + c;
-        float4 lo = make_float4(acc[u][0] * inv_len, acc[u][1] * inv_len, acc[u][2] * inv_len, acc[u][3] * inv_len);
-        float4 hi = make_float4(acc[u][4] * inv_len, acc[u][5] * inv_len, acc[u][6] * inv_len, acc[u][7] * inv_len);
-        reinterpret_cast<float4*>(dst)[0] = lo;
-        reinterpret_cast<float4*>(dst)[1] = hi;
+        const int64_t bh = static_cast<int64_t>(b) * a.heads + h;
+        if (which == 0) {  // Q: [B, heads, nblk, D]
+            float* dst = a.out[0] + (bh * a.nblk + blk) * D + c;
+            reinterpret_cast<float4*>(dst)[0] =
+                make_float4(acc[u][0] * inv_len, acc[u][1] * inv_len, acc[u][2] * inv_len, acc[u][3] * inv_len);
+            reinterpret_cast<float4*>(dst)[1] =
+                make_float4(acc[u][4] * inv_len, acc[u][5] * inv_len, acc[u][6] * inv_len, acc[u][7] * inv_len);
+        } else {  // K: channel-major [B, heads, D, kstride]
+            float* dst = a.out[1] + (bh * D + c) * kstride + blk;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) dst[static_cast<int64_t>(i) * kstride] = acc[u][i] * inv_len;
+        }
     }
 }
 
@@ -125,51 +135,74 @@ __device__ __forceinline__ uint32_t order_key(float f) {
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// grid: (ceil(nblk / 16), B*heads).  Dynamic shared memory:
-// qbar[16][96] fp32, scores[16][nblk] fp32, histograms[16][256] u32.
+// grid: (ceil(nblk / 16), B*heads), 512 threads.  Dynamic shared memory:
+// qbar[D][16] fp32 (the CTA's 16 query-block means, channel-major),
+// scores[16][nblk4] fp32 (nblk4 = nblk rounded up to 4), histograms[16][256] u32.
+//
+// Scores: thread t computes query blocks 8*(t/256) .. +7 against key blocks
+// j0 + 4*(t%256) .. +3, j0 = 0, 1024, ...: an 8 x 4 register tile.  Per
+// channel it reads its four key means with one 16-byte load -- the K means are
+// channel-major, so a warp's loads are 512 contiguous bytes -- and two 16-byte
+// broadcasts of the query means.  Every dot product adds q_c * k_c in channel
+// order c = 0..D-1 with one fmaf per channel, then scales by 1/sqrt(D).
 template <int D>
-__global__ void __launch_bounds__(kScoreThreads) score_topk_kernel(const ScoreArgs a) {
+__global__ void __launch_bounds__(kScoreThreads, 2) score_topk_kernel(const ScoreArgs a) {
     extern __shared__ __align__(16) float smem[];
-    float* qbar = smem;                                   // [16][96]
-    float* scores = qbar + kRowsPerCta * D;               // [16][nblk]
-    uint32_t* hist = reinterpret_cast<uint32_t*>(scores + kRowsPerCta * a.nblk);  // [16][256]
+    const int nblk4 = pooled_k_stride(a.nblk);
+    float* qbar = smem;                                                  // [D][16]
+    float* scores = qbar + kRowsPerCta * D;                              // [16][nblk4]
+    uint32_t* hist = reinterpret_cast<uint32_t*>(scores + kRowsPerCta * nblk4);  // [16][256]
 
     const int bh = blockIdx.y;
     const int i0 = blockIdx.x * kRowsPerCta;
     const int rows = min(kRowsPerCta, a.nblk - i0);
     const float* qsrc = a.qp + (static_cast<int64_t>(bh) * a.nblk + i0) * D;
-    const float* ksrc = a.kp + static_cast<int64_t>(bh) * a.nblk * D;
+    const float* ksrc = a.kp + static_cast<int64_t>(bh) * D * nblk4;
 
-    for (int e = threadIdx.x; e < kRowsPerCta * D; e += kScoreThreads)
-        qbar[e] = (e < rows * D) ? qsrc[e] : 0.f;
+    for (int e = threadIdx.x; e < kRowsPerCta * D; e += kScoreThreads) {
+        const int r = e / D, c = e - r * D;
+        qbar[c * kRowsPerCta + r] = (r < rows) ? qsrc[e] : 0.f;
+    }
     __syncthreads();
 
-    // scores[r][j] = (qbar_r . kbar_j) * inv_sqrt_d, dot in channel order
-    for (int j = threadIdx.x; j < a.nblk; j += kScoreThreads) {
-        float dot[kRowsPerCta];
+    const int rh = threadIdx.x >> 8;   // query blocks 8*rh .. 8*rh+7 of the CTA
+    const int kt = threadIdx.x & 255;  // key blocks j0 + 4*kt .. +3
+    for (int j0 = 0; j0 < nblk4; j0 += 1024) {
+        const int j = j0 + 4 * kt;
+        if (j >= nblk4) break;
+        float acc[8][4];
 #pragma unroll
-        for (int r = 0; r < kRowsPerCta; ++r) dot[r] = 0.f;
-        const float4* kj = reinterpret_cast<const float4*>(ksrc + static_cast<int64_t>(j) * D);
+        for (int r = 0; r < 8; ++r)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) acc[r][i] = 0.f;
+        const float* kc = ksrc + j;
 #pragma unroll 4
-        for (int c4 = 0; c4 < D / 4; ++c4) {
-            const float4 kv = __ldg(kj + c4);
+        for (int c = 0; c < D; ++c) {
+            const float4 kv = __ldg(reinterpret_cast<const float4*>(kc + static_cast<int64_t>(c) * nblk4));
+            const float4 qa = reinterpret_cast<const float4*>(qbar + c * kRowsPerCta + 8 * rh)[0];
+            const float4 qb = reinterpret_cast<const float4*>(qbar + c * kRowsPerCta + 8 * rh)[1];
+            const float q[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
 #pragma unroll
-            for (int r = 0; r < kRowsPerCta; ++r) {
-                const float4 qv = reinterpret_cast<const float4*>(qbar + r * D)[c4];
-                dot[r] = fmaf(qv.x, kv.x, dot[r]);
-                dot[r] = fmaf(qv.y, kv.y, dot[r]);
-                dot[r] = fmaf(qv.z, kv.z, dot[r]);
-                dot[r] = fmaf(qv.w, kv.w, dot[r]);
+            for (int r = 0; r < 8; ++r) {
+                acc[r][0] = fmaf(q[r], kv.x, acc[r][0]);
+                acc[r][1] = fmaf(q[r], kv.y, acc[r][1]);
+                acc[r][2] = fmaf(q[r], kv.z, acc[r][2]);
+                acc[r][3] = fmaf(q[r], kv.w, acc[r][3]);
             }
         }
+        // key blocks past nblk (the padding of the last group of four) are
+        // stored too and never read
 #pragma unroll
-        for (int r = 0; r < kRowsPerCta; ++r) scores[r * a.nblk + j] = dot[r] * a.inv_sqrt_d;
+        for (int r = 0; r < 8; ++r)
+            reinterpret_cast<float4*>(scores + (8 * rh + r) * nblk4 + j)[0] =
+                make_float4(acc[r][0] * a.inv_sqrt_d, acc[r][1] * a.inv_sqrt_d, acc[r][2] * a.inv_sqrt_d,
+                            acc[r][3] * a.inv_sqrt_d);
     }
     __syncthreads();
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (warp >= rows) return;
-    const float* s = scores + warp * a.nblk;
+    const float* s = scores + warp * nblk4;
     uint32_t* h = hist + warp * 256;
 
     // radix select of the kk-th largest key, 8 bits per pass, most significant first
@@ -245,7 +278,8 @@ __global__ void __launch_bounds__(kScoreThreads) score_topk_kernel(const ScoreAr
 }
 
 size_t score_smem_bytes(int nblk, int d) {
-    return (static_cast<size_t>(kRowsPerCta) * d + static_cast<size_t>(kRowsPerCta) * nblk) * sizeof(float) +
+    return (static_cast<size_t>(kRowsPerCta) * d + static_cast<size_t>(kRowsPerCta) * pooled_k_stride(nblk)) *
+               sizeof(float) +
            static_cast<size_t>(kRowsPerCta) * 256 * sizeof(uint32_t);
 }
 
@@ -291,7 +325,7 @@ cudaError_t pool(const void* q, const void* k, const Shape& s, int nblk, float* 
 
 int route_max_blocks(int d) {
     // largest nblk whose score tile fits the shared-memory budget
-    return static_cast<int>((kScoreSmemLimit - score_smem_bytes(0, d)) / (kRowsPerCta * sizeof(float)));
+    return static_cast<int>((kScoreSmemLimit - score_smem_bytes(0, d)) / (kRowsPerCta * sizeof(float))) & ~3;
 }
 
 cudaError_t launch_route_scores(const float* pooled_q, const float* pooled_k, const Shape& s, int nblk, int kk,

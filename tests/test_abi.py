@@ -58,13 +58,14 @@ def test_workspace_size():
     n = ctypes.c_size_t()
     d = _desc(N=124992)
     assert lib.h3a_route_workspace_size(ctypes.byref(d), 128, ctypes.byref(n)) == 0
-    nblk = 977
-    assert n.value == 2 * ((56 * nblk * 96 * 4 + 255) // 256 * 256)
+    nblk, nblk4 = 977, 980  # K's means are channel-major, rows of key blocks padded to a multiple of 4
+    a256 = lambda x: (x + 255) // 256 * 256
+    assert n.value == a256(56 * nblk * 96 * 4) + a256(56 * 96 * nblk4 * 4)
     assert lib.h3a_route_workspace_size(ctypes.byref(d), 64, ctypes.byref(n)) == 2  # block must be 128
     # 42 heads x 128 (the same 5376-wide hidden state): the router takes head_dim 128
     wide = _desc(N=124992, heads=42, D=128)
     assert lib.h3a_route_workspace_size(ctypes.byref(wide), 128, ctypes.byref(n)) == 0
-    assert n.value == 2 * ((42 * nblk * 128 * 4 + 255) // 256 * 256)
+    assert n.value == a256(42 * nblk * 128 * 4) + a256(42 * 128 * nblk4 * 4)
     bad = _desc(D=64)
     assert lib.h3a_route_workspace_size(ctypes.byref(bad), 128, ctypes.byref(n)) == 2
 

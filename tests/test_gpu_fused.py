@@ -34,13 +34,16 @@ CASES = [
 
 
 def _pooled_halves(ws: torch.Tensor, B: int, heads: int, nblk: int):
-    """The two fp32 [B, heads, nblk, 96] tensors of a router workspace."""
+    """The block means in a router workspace, both as fp32 [B, heads, nblk, 96]:
+    Q's are stored that way, K's channel-major ([B, heads, 96, nblk rounded up
+    to 4]) after Q's, on the next 256-byte boundary."""
     n = B * heads * nblk * 96
+    nblk4 = (nblk + 3) // 4 * 4
     half = (n * 4 + 255) // 256 * 256
     f = ws.view(torch.uint8)
     q = f[:n * 4].view(torch.float32).view(B, heads, nblk, 96)
-    k = f[half:half + n * 4].view(torch.float32).view(B, heads, nblk, 96)
-    return q, k
+    kt = f[half:half + B * heads * 96 * nblk4 * 4].view(torch.float32).view(B, heads, 96, nblk4)
+    return q, kt[..., :nblk].transpose(2, 3)
 
 
 def _pool_bound(orc, out_bits: np.ndarray) -> np.ndarray:
