@@ -135,6 +135,46 @@ __device__ __forceinline__ uint32_t order_key(float f) {
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// Given a 256-bin histogram h (bin 255 the largest values) and a rank
+// 1 <= r <= total, finds the bin holding the r-th largest value and the
+// number of values in the bins above it.  Warp-collective; lane l reads bins
+// 255-8l .. 248-8l and the counts are prefix-summed across the warp.
+__device__ __forceinline__ void select_digit(const uint32_t* h, int lane, uint32_t r, uint32_t& bin,
+                                             uint32_t& above) {
+    uint32_t cnt[8];
+    uint32_t local = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        cnt[i] = h[255 - (lane * 8 + i)];
+        local += cnt[i];
+    }
+    uint32_t incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+    }
+    const uint32_t excl = incl - local;  // values in larger bins, from lanes before
+    const bool mine = excl < r && r <= incl;
+    const uint32_t owner = __ballot_sync(0xffffffffu, mine);
+    const int src = __ffs(owner) - 1;
+    uint32_t b = 0, ab = 0;
+    if (mine) {
+        uint32_t run = excl;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            if (run < r && r <= run + cnt[i]) {
+                b = 255 - (lane * 8 + i);
+                ab = run;
+                break;
+            }
+            run += cnt[i];
+        }
+    }
+    bin = __shfl_sync(0xffffffffu, b, src);
+    above = __shfl_sync(0xffffffffu, ab, src);
+}
+
 // grid: (ceil(nblk / 16), B*heads), 512 threads.  Dynamic shared memory:
 // qbar[D][16] fp32 (the CTA's 16 query-block means, channel-major),
 // scores[16][nblk4] fp32 (nblk4 = nblk rounded up to 4), histograms[16][256] u32.
@@ -204,6 +244,78 @@ __global__ void __launch_bounds__(kScoreThreads, 2) score_topk_kernel(const Scor
     if (warp >= rows) return;
     const float* s = scores + warp * nblk4;
     uint32_t* h = hist + warp * 256;
+    int32_t* out = a.idx + (static_cast<int64_t>(bh) * a.nblk + i0 + warp) * a.kk;
+    const uint32_t lt_mask = (1u << lane) - 1u;
+
+    // Selection of the kk highest scores of the row, ties to the lower index,
+    // emitted ascending.  Fast path: 256 buckets linear in the score between
+    // the row's min and max.  The bucket index is a non-decreasing function of
+    // the value, so every key in a higher bucket is strictly larger than every
+    // key in a lower one and equal values share a bucket; the buckets above
+    // the one holding the kk-th largest are taken whole, and the `need` best
+    // of that bucket by (score descending, index ascending) are ranked exactly
+    // -- the same set the radix select below finds.  The radix select runs
+    // when that bucket holds more than 32 keys or the row is constant.
+    float smax = -INFINITY, smin = INFINITY;
+    for (int j = lane; j < a.nblk; j += 32) {
+        const float v = s[j];
+        smax = fmaxf(smax, v);
+        smin = fminf(smin, v);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, o));
+        smin = fminf(smin, __shfl_xor_sync(0xffffffffu, smin, o));
+    }
+    const float scale = 256.0f / (smax - smin);
+    if (smax > smin && scale < INFINITY) {
+        auto bucket = [&](float v) { return min(255, static_cast<int>((v - smin) * scale)); };
+#pragma unroll
+        for (int i = 0; i < 8; ++i) h[lane * 8 + i] = 0u;
+        __syncwarp();
+        for (int j = lane; j < a.nblk; j += 32) atomicAdd(&h[bucket(s[j])], 1u);
+        __syncwarp();
+        uint32_t bstar, above;
+        select_digit(h, lane, static_cast<uint32_t>(a.kk), bstar, above);
+        const int need = a.kk - static_cast<int>(above);  // 1 .. size of bucket bstar
+        __syncwarp();
+        // the bucket's keys, in index order, into h[0 .. 31]
+        int cnt = 0;
+        for (int base = 0; base < a.nblk; base += 32) {
+            const int j = base + lane;
+            const bool c = j < a.nblk && bucket(s[j]) == static_cast<int>(bstar);
+            const uint32_t m = __ballot_sync(0xffffffffu, c);
+            const int pos = cnt + __popc(m & lt_mask);
+            if (c && pos < 32) h[pos] = static_cast<uint32_t>(j);
+            cnt += __popc(m);
+        }
+        __syncwarp();
+        if (cnt <= 32) {
+            const int cj = lane < cnt ? static_cast<int>(h[lane]) : 0;
+            const float cs = lane < cnt ? s[cj] : -INFINITY;
+            int rank = 0;  // candidates ahead of this one in (score desc, index asc)
+            for (int m = 0; m < cnt; ++m) {
+                const float sm = __shfl_sync(0xffffffffu, cs, m);
+                const int jm = __shfl_sync(0xffffffffu, cj, m);
+                rank += (sm > cs || (sm == cs && jm < cj)) ? 1 : 0;
+            }
+            const uint32_t take = __ballot_sync(0xffffffffu, lane < cnt && rank < need);
+            int written = 0, eq_seen = 0;
+            for (int base = 0; base < a.nblk; base += 32) {
+                const int j = base + lane;
+                const int bk = j < a.nblk ? bucket(s[j]) : -1;
+                const bool eq = bk == static_cast<int>(bstar);
+                const uint32_t eq_mask = __ballot_sync(0xffffffffu, eq);
+                const bool sel = bk > static_cast<int>(bstar) ||
+                                 (eq && ((take >> (eq_seen + __popc(eq_mask & lt_mask))) & 1u));
+                const uint32_t sel_mask = __ballot_sync(0xffffffffu, sel);
+                if (sel) out[written + __popc(sel_mask & lt_mask)] = j;
+                written += __popc(sel_mask);
+                eq_seen += __popc(eq_mask);
+            }
+            return;
+        }
+    }
 
     // radix select of the kk-th largest key, 8 bits per pass, most significant first
     uint32_t prefix = 0;
@@ -218,39 +330,8 @@ __global__ void __launch_bounds__(kScoreThreads, 2) score_topk_kernel(const Scor
             if ((u & hi_mask) == (prefix & hi_mask)) atomicAdd(&h[(u >> shift) & 255u], 1u);
         }
         __syncwarp();
-        // lane l owns digits 255-8l .. 248-8l (descending)
-        uint32_t cnt[8];
-        uint32_t local = 0;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            cnt[i] = h[255 - (lane * 8 + i)];
-            local += cnt[i];
-        }
-        uint32_t incl = local;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += t;
-        }
-        const uint32_t excl = incl - local;  // keys with a larger digit, from lanes before
-        const bool mine = excl < static_cast<uint32_t>(remaining) && static_cast<uint32_t>(remaining) <= incl;
-        const uint32_t owner = __ballot_sync(0xffffffffu, mine);
-        const int src = __ffs(owner) - 1;
-        uint32_t digit = 0, above = 0;
-        if (mine) {
-            uint32_t run = excl;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                if (run < static_cast<uint32_t>(remaining) && static_cast<uint32_t>(remaining) <= run + cnt[i]) {
-                    digit = 255 - (lane * 8 + i);
-                    above = run;
-                    break;
-                }
-                run += cnt[i];
-            }
-        }
-        digit = __shfl_sync(0xffffffffu, digit, src);
-        above = __shfl_sync(0xffffffffu, above, src);
+        uint32_t digit, above;
+        select_digit(h, lane, static_cast<uint32_t>(remaining), digit, above);
         prefix |= digit << shift;
         remaining -= static_cast<int>(above);
         __syncwarp();
@@ -258,8 +339,6 @@ __global__ void __launch_bounds__(kScoreThreads, 2) score_topk_kernel(const Scor
 
     // emit: every key above the threshold, plus the first `remaining` keys equal
     // to it (lowest indices first), in ascending index order
-    int32_t* out = a.idx + (static_cast<int64_t>(bh) * a.nblk + i0 + warp) * a.kk;
-    const uint32_t lt_mask = (1u << lane) - 1u;
     int written = 0, eq_seen = 0;
     for (int base = 0; base < a.nblk; base += 32) {
         const int j = base + lane;
