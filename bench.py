@@ -643,6 +643,43 @@ def cpu_baseline(d, w, nrows):
                       f"{dt:.1f} s"}
 
 
+def run_router_only(args, local):
+    """Scores + top-k alone (h3a_route_pooled) on seeded random block means of
+    the workload's shape -- a small case for profilers: about 42 MB on the
+    device at 124,992 tokens instead of the full step's tensors.  Prints one
+    JSON line with the mean time of --steps calls after --warmup calls."""
+    import rope_block_sparse_b200 as h3a
+    from rope_block_sparse_b200 import synth
+
+    w = synth.WORKLOADS[args.workload]
+    if w.head_dim != 96:
+        raise SystemExit("--kernel-only router takes a head_dim-96 workload (the pooled router's width)")
+    dev = torch.device("cuda", local)
+    D, nblk = w.head_dim, (w.N + 127) // 128
+    # q only supplies the shape: the router reads the block means in the workspace
+    q = torch.empty((w.N + w.heads) * D, dtype=torch.bfloat16, device=dev).as_strided(
+        (w.B, w.N, w.heads, D), (0, D, D, 1))
+    ws = torch.empty(h3a.route_workspace_size(q), dtype=torch.uint8, device=dev)
+    g = torch.Generator(device=dev).manual_seed(0)
+    ws.view(torch.float32).copy_(0.3 * torch.randn(ws.numel() // 4, generator=g, device=dev))
+    sparsity = w.sparsity if w.sparsity else SPARSITY
+    blocks = torch.empty((w.B, w.heads, nblk, h3a.route_k(nblk, sparsity)), dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        h3a.route_pooled(q, sparsity, ws, out=blocks)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(args.steps):
+        h3a.route_pooled(q, sparsity, ws, out=blocks)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return {"kernel": "score_topk_kernel (h3a_route_pooled)",
+            "workload": f"{w.name}: seeded N(0, 0.3^2) block means of {w.B} x {w.heads} heads x {nblk} blocks x {D}, "
+                        f"sparsity {sparsity} (k = {blocks.shape[-1]})",
+            "ms": round(e0.elapsed_time(e1) / args.steps, 4), "steps": args.steps, "warmup": args.warmup}
+
+
 def run_reference(args, rank, world):
     """Reference arm: the fp64 oracle on the host cores, each step a bounded sample."""
     if rank != 0:
@@ -698,6 +735,8 @@ def main():
     ap.add_argument("--ref-rows", type=int, default=128, help="query rows per reference-arm step")
     ap.add_argument("--no-video10s", dest="video10s", action="store_false",
                     help="skip the 245,952-token pass reported beside the headline")
+    ap.add_argument("--kernel-only", choices=["router"], default=None,
+                    help="time one kernel alone on a small case for profilers (one GPU): router = scores + top-k")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -707,6 +746,10 @@ def main():
         line = run_reference(args, rank, world)
         if line is not None:
             print(json.dumps(line), flush=True)
+        return
+    if args.kernel_only == "router":
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        print(json.dumps(run_router_only(args, int(os.environ.get("LOCAL_RANK", "0")))), flush=True)
         return
     rank, world, local = dist_setup(args.gpus)
     try:
