@@ -154,7 +154,9 @@ h3a_status h3a_route(const void* q, const void* k, const h3a_qkv_desc* d, double
  *             16-B aligned, owned by the caller; it must not overlap q, k,
  *             q_out or k_out.
  * Other arguments, layouts and errors: as h3a_qk_norm_rope; WORKSPACE if the
- * workspace is null, misaligned or too small; UNSUPPORTED if B > 65535. */
+ * workspace is null, misaligned or too small; UNSUPPORTED if B > 65535.  Q
+ * and K stream through shared memory with TMA; a bounded pipeline wait that
+ * expired is reported by h3a_last_device_error (H3A_ERR_TIMEOUT). */
 h3a_status h3a_qk_norm_rope_pool(const void* q, const void* k, const h3a_qkv_desc* d,
                                  const float* gamma_q, const float* gamma_k, h3a_grid grid,
                                  double theta, float eps, void* q_out, void* k_out,

@@ -104,7 +104,11 @@ size_t pooled_k_bytes(const Shape& s, int nblk) {
 
 }  // namespace
 
-cudaError_t make_qkv_tensor_map(CUtensorMap* map, const void* base, const Shape& s) {
+namespace {
+// Tiled tensor map over a [B, N, heads, d] bf16 tensor (d contiguous) with the
+// given box and swizzle; elements outside the tensor read as zero.
+cudaError_t encode_qkv_map(CUtensorMap* map, const void* base, const Shape& s, const cuuint32_t (&box)[4],
+                           CUtensorMapSwizzle swizzle) {
     std::call_once(g_encode_once, []() {
         void* fn = nullptr;
         cudaDriverEntryPointQueryResult q;
@@ -118,12 +122,22 @@ cudaError_t make_qkv_tensor_map(CUtensorMap* map, const void* base, const Shape&
     // byte strides of dims 1..3; a size-1 dim gets a nominal (unused) stride
     auto stride_or = [](int64_t st, int64_t fallback) { return static_cast<cuuint64_t>((st > 0 ? st : fallback) * 2); };
     const cuuint64_t strides[3] = {stride_or(s.sh, s.d), stride_or(s.sn, s.d), stride_or(s.sb, s.d)};
-    const cuuint32_t box[4] = {32, 1, 128, 1};
     const cuuint32_t elem_strides[4] = {1, 1, 1, 1};
     CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
-                          elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
-                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                          elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+}  // namespace
+
+cudaError_t make_qkv_tensor_map(CUtensorMap* map, const void* base, const Shape& s) {
+    const cuuint32_t box[4] = {32, 1, 128, 1};
+    return encode_qkv_map(map, base, s, box, CU_TENSOR_MAP_SWIZZLE_64B);
+}
+
+cudaError_t make_head_slice_tensor_map(CUtensorMap* map, const void* base, const Shape& s) {
+    const cuuint32_t box[4] = {static_cast<cuuint32_t>(kHeadDim), static_cast<cuuint32_t>(kPrologueSliceHeads), 1, 1};
+    return encode_qkv_map(map, base, s, box, CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
 }  // namespace h3a
@@ -259,14 +273,21 @@ h3a_status h3a_qk_norm_rope_pool(const void* q, const void* k, const h3a_qkv_des
     h3a_status rc = prologue_check(q, k, d, gamma_q, gamma_k, grid, theta, eps, q_out, k_out, &s);
     if (rc != H3A_OK) return rc;
     const int nblk = (s.N + kBlock - 1) / kBlock;
-    if (s.B > 65535 || (s.heads + 27) / 28 > 65535) return H3A_ERR_UNSUPPORTED;
+    if (s.B > 65535 || (s.heads + kPrologueSliceHeads - 1) / kPrologueSliceHeads > 65535) return H3A_ERR_UNSUPPORTED;
     const size_t half = pooled_q_bytes(s, nblk);
     if (workspace == nullptr || !aligned16(workspace) || ws_bytes < half + pooled_k_bytes(s, nblk))
         return H3A_ERR_WORKSPACE;
     float* pq = static_cast<float*>(workspace);
     float* pk = reinterpret_cast<float*>(static_cast<char*>(workspace) + half);
-    cudaError_t e = launch_qk_norm_rope_pool(q, k, q_out, k_out, gamma_q, gamma_k, s, grid.H, grid.W, theta, eps, pq,
-                                             pk, reinterpret_cast<cudaStream_t>(stream));
+    int* status = nullptr;
+    rc = status_word(&status);
+    if (rc != H3A_OK) return rc;
+    CUtensorMap tq, tk;
+    cudaError_t e = make_head_slice_tensor_map(&tq, q, s);
+    if (e == cudaSuccess) e = make_head_slice_tensor_map(&tk, k, s);
+    if (e != cudaSuccess) return cuda_fail(e);
+    e = launch_qk_norm_rope_pool(tq, tk, q_out, k_out, gamma_q, gamma_k, s, grid.H, grid.W, theta, eps, pq, pk,
+                                 status, kWaitLimitNs, reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? H3A_OK : cuda_fail(e);
 }
 

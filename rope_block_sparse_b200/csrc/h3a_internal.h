@@ -32,10 +32,15 @@ cudaError_t launch_qk_fullnorm_rope(const void* q, const void* k, void* q_out, v
                                     cudaStream_t st);
 
 // Prologue that also writes the fp32 means of its rounded outputs over
-// 128-token blocks into pool_q / pool_k (the router's layouts, below) (prologue.cu).
-cudaError_t launch_qk_norm_rope_pool(const void* q, const void* k, void* q_out, void* k_out, const float* gamma_q,
-                                     const float* gamma_k, const Shape& s, int H, int W, double theta, float eps,
-                                     float* pool_q, float* pool_k, cudaStream_t st);
+// 128-token blocks into pool_q / pool_k (the router's layouts, below)
+// (prologue.cu).  Q and K are read through tensor maps made by
+// make_head_slice_tensor_map; a bounded wait that expires sets `status`.
+cudaError_t launch_qk_norm_rope_pool(const CUtensorMap& tq, const CUtensorMap& tk, void* q_out, void* k_out,
+                                     const float* gamma_q, const float* gamma_k, const Shape& s, int H, int W,
+                                     double theta, float eps, float* pool_q, float* pool_k, int* status,
+                                     uint64_t timeout_ns, cudaStream_t st);
+// Heads per slice of the tensor map the prologue with pooling reads.
+constexpr int kPrologueSliceHeads = 28;
 
 // The router's fp32 block means: Q's as [B, heads, nblk, d]; K's channel-major,
 // [B, heads, d, pooled_k_stride(nblk)] (one 16-byte-aligned row of key blocks
@@ -77,5 +82,9 @@ cudaError_t launch_selftest_mma(const CUtensorMap& ta, const CUtensorMap& tb, fl
 // Tensor map over a [B, N, heads, 96] bf16 tensor with a {32, 1, 128, 1} box,
 // 64-byte swizzle (h3a_api.cu).
 cudaError_t make_qkv_tensor_map(CUtensorMap* map, const void* base, const Shape& s);
+// Tensor map over the same tensor with a {96, kPrologueSliceHeads, 1, 1} box:
+// one token's slice of consecutive heads, no swizzle, heads past the tensor
+// read as zero (h3a_api.cu).
+cudaError_t make_head_slice_tensor_map(CUtensorMap* map, const void* base, const Shape& s);
 
 }  // namespace h3a

@@ -18,6 +18,7 @@
 #include <cmath>
 
 #include "h3a_internal.h"
+#include "sm100.cuh"
 
 namespace h3a {
 namespace {
@@ -42,10 +43,12 @@ struct PrologueArgs {
     // theta^(-2j/32) as an unevaluated sum hi + lo of two floats
     float freq_hi[kPairsPerSection];
     float freq_lo[kPairsPerSection];
-    // block pooling (qk_norm_rope_pool_kernel only): fp32 [B, heads, nblk, 96]
+    // block pooling (qk_norm_rope_pool_kernel only): the router's fp32 means
     float* pool_q;
     float* pool_k;
     int nblk;
+    int* status;          // device status word (bounded-wait timeouts)
+    uint64_t timeout_ns;  // limit of one pipeline wait
 };
 
 __device__ __forceinline__ void unpack4(uint2 v, float* x) {
@@ -187,26 +190,38 @@ __global__ void __launch_bounds__(kThreads, 3) qk_norm_rope_kernel(const Prologu
 // produces those means while the rounded outputs are still in registers, so
 // the router need not read Q and K back from HBM.
 //
-// One CTA per (batch, 128-token block, chunk of 28 heads); warp w owns heads
-// 28*chunk + 4w .. +3 with the prologue's lane layout (8 lanes per head, 12
-// channels per lane) and walks the block's tokens in order.  Each (head,
-// channel) sum therefore lives in one lane and adds the bf16-rounded outputs
-// in token order, exactly as the separate pooling kernel does, so the means
-// are bit-identical to it.  The rotation of every (token, pair) of the block
-// is computed once per CTA into shared memory: a warp now covers 4 heads per
-// token instead of 56, and computing the rotation per warp would cost more
-// issue slots than the HBM-bound prologue has to spare.  Each warp keeps the
-// loads of four tokens in flight (128 registers, two CTAs per SM): with one
-// token per iteration the kernel reached only a third of HBM bandwidth.
-constexpr int kPoolWarps = 7;
-constexpr int kPoolThreads = 32 * kPoolWarps;              // 224
+// One CTA per (batch, 128-token block, chunk of 28 heads).  Warp 7 streams the
+// block's token rows into a ring of kPoolRing slots in shared memory with TMA
+// (one 28-head x 96-channel slice of Q and one of K per token, 5,376 bytes
+// each, through a tensor map, so any head and token stride works), so the
+// loads in flight hold no registers.  Warps 0-6 own four heads each with the
+// prologue's lane layout (8 lanes per head, 12 channels per lane): per token a
+// warp reads its slice from the slot, releases the slot, normalises, rotates,
+// stores the rounded outputs and adds them to its block sums.  Each (head,
+// channel) sum lives in one lane and adds the bf16-rounded outputs in token
+// order, exactly as the separate pooling kernel does, so the means are
+// bit-identical to it.  The rotation of every (token, pair) of the block is
+// computed once per CTA into shared memory (while the first tokens load): a
+// warp covers 4 heads per token instead of 56, and computing the rotation per
+// warp would cost more issue slots than the HBM-bound prologue has to spare.
+// Every barrier wait is bounded; an expired wait sets the device status word.
+constexpr int kPoolWarps = 7;                              // consumer warps
+constexpr int kPoolThreads = 32 * (kPoolWarps + 1);        // + the TMA producer warp
+constexpr int kPoolConsumers = 32 * kPoolWarps;            // 224
 constexpr int kPoolHeadsPerCta = 4 * kPoolWarps;           // 28
 constexpr int kPairsPerHead = kHeadDim / 2;                // 48
-constexpr size_t kPoolSmemBytes = sizeof(float2) * kBlock * kPairsPerHead;  // 48 KB
-#ifndef H3A_POOL_UNROLL
-#define H3A_POOL_UNROLL 4
-#endif
-constexpr int kPoolUnroll = H3A_POOL_UNROLL;  // tokens whose loads are in flight together
+constexpr int kPoolRing = 5;                               // tokens in flight per CTA
+constexpr int kSliceBytes = kPoolHeadsPerCta * kHeadDim * 2;  // 5,376
+static_assert(kSliceBytes % 128 == 0, "slots stay 128-byte aligned");
+
+struct PoolSmem {
+    uint8_t ring[kPoolRing][2][kSliceBytes];     // [slot][Q, K][28 heads x 96 bf16]
+    float2 rot[kBlock * kPairsPerHead];          // (cos, sin) per (token, pair)
+    uint64_t full[kPoolRing], empty[kPoolRing];
+    int abort_flag;
+    int never;  // stays 0: abort flag for the producer's final drain
+};
+constexpr size_t kPoolSmemBytes = sizeof(PoolSmem) + 1024;  // + alignment slack
 
 __device__ __forceinline__ void add_rounded(const uint32_t (&out)[kPairsPerLane], float (&acc)[kChanPerLane]) {
 #pragma unroll
@@ -216,25 +231,81 @@ __device__ __forceinline__ void add_rounded(const uint32_t (&out)[kPairsPerLane]
     }
 }
 
-__global__ void __launch_bounds__(kPoolThreads, 2) qk_norm_rope_pool_kernel(const PrologueArgs a) {
-    extern __shared__ float2 rot[];  // [kBlock][kPairsPerHead]: (cos, sin)
+__device__ __forceinline__ void pool_timeout(const PrologueArgs& a, volatile int* abort_flag) {
+    *abort_flag = 1;
+    atomicOr(a.status, kDevTimeout);
+}
+
+__global__ void __launch_bounds__(kPoolThreads, 2)
+    qk_norm_rope_pool_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                             const PrologueArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t base_addr = smem_u32(smem_raw);
+    PoolSmem& sm = *reinterpret_cast<PoolSmem*>(smem_raw + (((base_addr + 1023u) & ~1023u) - base_addr));
     const int blk = blockIdx.x, b = blockIdx.y, chunk = blockIdx.z;
     const int n0 = blk * kBlock;
     const int len = min(a.N - n0, kBlock);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    volatile int* abort_flag = &sm.abort_flag;
 
-    for (int e = threadIdx.x; e < len * kPairsPerHead; e += kPoolThreads) {
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kPoolRing; ++i) {
+            mbar_init(&sm.full[i], 1);
+            mbar_init(&sm.empty[i], kPoolWarps);  // one arrival per consumer warp
+        }
+        sm.abort_flag = 0;
+        sm.never = 0;
+        fence_barrier_init();
+    }
+    __syncthreads();
+
+    if (warp == kPoolWarps) {
+        // TMA producer: token t goes to slot t % kPoolRing once the consumers
+        // have released that slot's previous token
+        if (lane == 0) {
+            prefetch_tensor_map(&tq);
+            prefetch_tensor_map(&tk);
+            const int h0 = chunk * kPoolHeadsPerCta;
+            int issued = 0;
+            for (int t = 0; t < len; ++t) {
+                const int slot = t % kPoolRing;
+                const uint32_t ph = static_cast<uint32_t>(t / kPoolRing) & 1u;
+                if (t >= kPoolRing && !mbar_wait(&sm.empty[slot], ph ^ 1u, abort_flag, a.timeout_ns)) {
+                    pool_timeout(a, abort_flag);
+                    break;
+                }
+                // the consumers read the slot's previous token with ordinary
+                // shared-memory loads; the TMA refill below writes through the
+                // async proxy, which the barrier alone does not order after them
+                fence_proxy_async_shared();
+                mbar_arrive_expect_tx(&sm.full[slot], 2 * kSliceBytes);
+                tma_load_4d(sm.ring[slot][0], &tq, &sm.full[slot], 0, h0, n0 + t, b);
+                tma_load_4d(sm.ring[slot][1], &tk, &sm.full[slot], 0, h0, n0 + t, b);
+                issued = t + 1;
+            }
+            // every load issued must have landed before the CTA exits (normally
+            // the consumers have already waited for each of them)
+            for (int t = max(0, issued - kPoolRing); t < issued; ++t)
+                mbar_wait(&sm.full[t % kPoolRing], static_cast<uint32_t>(t / kPoolRing) & 1u, &sm.never,
+                          a.timeout_ns);
+        }
+        return;
+    }
+
+    // consumers: the block's rotations first, while the first tokens load
+    for (int e = threadIdx.x; e < len * kPairsPerHead; e += kPoolConsumers) {
         const int i = e / kPairsPerHead, pair = e - i * kPairsPerHead;
         const int n = n0 + i;
         float c, sn;
         rotation(n / (a.H * a.W), (n / a.W) % a.H, n % a.W, pair, a.freq_hi, a.freq_lo, c, sn);
-        rot[e] = make_float2(c, sn);
+        sm.rot[e] = make_float2(c, sn);
     }
-    __syncthreads();
+    asm volatile("bar.sync 1, %0;" ::"n"(kPoolConsumers) : "memory");  // the consumer warps only
 
-    const int lane = threadIdx.x & 31;
     const int sub = lane & 7;
     const int c0 = sub * kChanPerLane;
-    const int h = chunk * kPoolHeadsPerCta + (threadIdx.x >> 5) * 4 + (lane >> 3);
+    const int hl = warp * 4 + (lane >> 3);  // head within the chunk
+    const int h = chunk * kPoolHeadsPerCta + hl;
     const bool active = h < a.heads;
     float gq[kChanPerLane], gk[kChanPerLane];
 #pragma unroll
@@ -247,36 +318,40 @@ __global__ void __launch_bounds__(kPoolThreads, 2) qk_norm_rope_pool_kernel(cons
     for (int i = 0; i < kChanPerLane; ++i) accq[i] = acck[i] = 0.f;
 
     const int64_t base = static_cast<int64_t>(b) * a.sb + static_cast<int64_t>(h) * a.sh + c0;
-    // kPoolUnroll tokens per iteration, all their loads issued first; the
-    // sums still add the tokens in order
-    for (int i = 0; i < len; i += kPoolUnroll) {
-        uint2 rq[kPoolUnroll][3], rk[kPoolUnroll][3];
-#pragma unroll
-        for (int u = 0; u < kPoolUnroll; ++u) {
-            const int64_t off = base + static_cast<int64_t>(n0 + i + u) * a.sn;
-            const bool act = active && i + u < len;
-            load3(a.q + off, act, rq[u]);
-            load3(a.k + off, act, rk[u]);
+    const int lane_off = hl * kHeadDim * 2 + sub * kChanPerLane * 2;  // byte offset of the lane's 12 channels
+    bool ok = true;
+    for (int t = 0; t < len; ++t) {
+        const int slot = t % kPoolRing;
+        const uint32_t ph = static_cast<uint32_t>(t / kPoolRing) & 1u;
+        if (!__all_sync(0xffffffffu, mbar_wait(&sm.full[slot], ph, abort_flag, a.timeout_ns))) {
+            ok = false;
+            break;
         }
+        const uint2* sq = reinterpret_cast<const uint2*>(sm.ring[slot][0] + lane_off);
+        const uint2* sk = reinterpret_cast<const uint2*>(sm.ring[slot][1] + lane_off);
+        const uint2 rq[3] = {sq[0], sq[1], sq[2]};
+        const uint2 rk[3] = {sk[0], sk[1], sk[2]};
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.empty[slot]);  // the slice is in registers
+        float cs[kPairsPerLane], sn[kPairsPerLane];
 #pragma unroll
-        for (int u = 0; u < kPoolUnroll; ++u) {
-            if (i + u >= len) break;
-            float cs[kPairsPerLane], sn[kPairsPerLane];
-#pragma unroll
-            for (int p = 0; p < kPairsPerLane; ++p) {
-                const float2 v = rot[(i + u) * kPairsPerHead + sub * kPairsPerLane + p];
-                cs[p] = v.x;
-                sn[p] = v.y;
-            }
-            const int64_t off = base + static_cast<int64_t>(n0 + i + u) * a.sn;
-            uint32_t oq[kPairsPerLane], ok[kPairsPerLane];
-            norm_rope(rq[u], gq, cs, sn, a.eps, oq);
-            norm_rope(rk[u], gk, cs, sn, a.eps, ok);
-            store3(oq, active, a.qo + off);
-            store3(ok, active, a.ko + off);
-            add_rounded(oq, accq);
-            add_rounded(ok, acck);
+        for (int p = 0; p < kPairsPerLane; ++p) {
+            const float2 v = sm.rot[t * kPairsPerHead + sub * kPairsPerLane + p];
+            cs[p] = v.x;
+            sn[p] = v.y;
         }
+        const int64_t off = base + static_cast<int64_t>(n0 + t) * a.sn;
+        uint32_t oq[kPairsPerLane], ok_[kPairsPerLane];
+        norm_rope(rq, gq, cs, sn, a.eps, oq);
+        norm_rope(rk, gk, cs, sn, a.eps, ok_);
+        store3(oq, active, a.qo + off);
+        store3(ok_, active, a.ko + off);
+        add_rounded(oq, accq);
+        add_rounded(ok_, acck);
+    }
+    if (!ok) {
+        pool_timeout(a, abort_flag);
+        return;
     }
     if (!active) return;
     const float inv_len = 1.0f / static_cast<float>(len);
@@ -443,12 +518,13 @@ cudaError_t launch_qk_norm_rope(const void* q, const void* k, void* q_out, void*
     return cudaGetLastError();
 }
 
-cudaError_t launch_qk_norm_rope_pool(const void* q, const void* k, void* q_out, void* k_out, const float* gamma_q,
-                                     const float* gamma_k, const Shape& s, int H, int W, double theta, float eps,
-                                     float* pool_q, float* pool_k, cudaStream_t st) {
+cudaError_t launch_qk_norm_rope_pool(const CUtensorMap& tq, const CUtensorMap& tk, void* q_out, void* k_out,
+                                     const float* gamma_q, const float* gamma_k, const Shape& s, int H, int W,
+                                     double theta, float eps, float* pool_q, float* pool_k, int* status,
+                                     uint64_t timeout_ns, cudaStream_t st) {
     PrologueArgs a;
-    a.q = static_cast<const __nv_bfloat16*>(q);
-    a.k = static_cast<const __nv_bfloat16*>(k);
+    a.q = nullptr;  // read through the tensor maps
+    a.k = nullptr;
     a.qo = static_cast<__nv_bfloat16*>(q_out);
     a.ko = static_cast<__nv_bfloat16*>(k_out);
     a.gq = gamma_q;
@@ -466,11 +542,13 @@ cudaError_t launch_qk_norm_rope_pool(const void* q, const void* k, void* q_out, 
     a.pool_q = pool_q;
     a.pool_k = pool_k;
     a.nblk = (s.N + kBlock - 1) / kBlock;
+    a.status = status;
+    a.timeout_ns = timeout_ns;
     const int chunks = (s.heads + kPoolHeadsPerCta - 1) / kPoolHeadsPerCta;
     cudaError_t e = cudaFuncSetAttribute(qk_norm_rope_pool_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(kPoolSmemBytes));
     if (e != cudaSuccess) return e;
-    qk_norm_rope_pool_kernel<<<dim3(a.nblk, s.B, chunks), kPoolThreads, kPoolSmemBytes, st>>>(a);
+    qk_norm_rope_pool_kernel<<<dim3(a.nblk, s.B, chunks), kPoolThreads, kPoolSmemBytes, st>>>(tq, tk, a);
     return cudaGetLastError();
 }
 

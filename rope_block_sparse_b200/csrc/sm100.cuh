@@ -80,6 +80,15 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
 
 // ---------------------------------------------------------------- TMA
 
+// Orders this thread's view of prior shared-memory accesses made through the
+// generic proxy (ordinary loads and stores, including other threads' accesses
+// it has synchronised with) before its subsequent async-proxy operations on
+// shared memory, e.g. a TMA load that overwrites a buffer other threads have
+// just read.
+__device__ __forceinline__ void fence_proxy_async_shared() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 __device__ __forceinline__ void prefetch_tensor_map(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
