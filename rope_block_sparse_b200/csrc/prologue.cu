@@ -107,16 +107,13 @@ __device__ __forceinline__ void norm_rope_store(const uint2 (&raw)[3], const flo
     store3(out, active, dst);
 }
 
-// cos / sin of the rotation of pair `pair` (0..47 within a head: section
-// pair / 16, index j = pair % 16) at grid position pos: fp32 sincos of the high
-// part of the angle pos * theta^(-2j/32), corrected to first order by its low
-// part (the frequency is an unevaluated sum hi + lo of two floats).
-__device__ __forceinline__ void rotation(int pt, int ph, int pw, int pair, const float* freq_hi,
-                                         const float* freq_lo, float& c_out, float& s_out) {
-    const int axis = pair / kPairsPerSection;
-    const int j = pair % kPairsPerSection;
-    // selects, not an indexed array: axis depends on the lane
-    const float ps = static_cast<float>(axis == 0 ? pt : (axis == 1 ? ph : pw));
+// cos / sin of the angle pos * theta^(-2j/32) of pair j of a section at axis
+// position `pos`: fp32 sincos of the high part of the angle, corrected to
+// first order by its low part (the frequency is an unevaluated sum hi + lo of
+// two floats).
+__device__ __forceinline__ void rotation_at(int pos, int j, const float* freq_hi, const float* freq_lo,
+                                            float& c_out, float& s_out) {
+    const float ps = static_cast<float>(pos);
     const float hi = freq_hi[j];
     const float a_hi = ps * hi;
     const float a_lo = fmaf(ps, hi, -a_hi) + ps * freq_lo[j];
@@ -124,6 +121,15 @@ __device__ __forceinline__ void rotation(int pt, int ph, int pw, int pair, const
     sincosf(a_hi, &s, &c);
     c_out = fmaf(-a_lo, s, c);
     s_out = fmaf(a_lo, c, s);
+}
+
+// The rotation of pair `pair` (0..47 within a head: section pair / 16 --
+// t, h, w -- index j = pair % 16) at grid position (pt, ph, pw).
+__device__ __forceinline__ void rotation(int pt, int ph, int pw, int pair, const float* freq_hi,
+                                         const float* freq_lo, float& c_out, float& s_out) {
+    const int axis = pair / kPairsPerSection;
+    // selects, not an indexed array: axis depends on the lane
+    rotation_at(axis == 0 ? pt : (axis == 1 ? ph : pw), pair % kPairsPerSection, freq_hi, freq_lo, c_out, s_out);
 }
 
 __device__ __forceinline__ void load3(const __nv_bfloat16* src, bool active, uint2 (&raw)[3]) {
@@ -200,10 +206,12 @@ __global__ void __launch_bounds__(kThreads, 3) qk_norm_rope_kernel(const Prologu
 // stores the rounded outputs and adds them to its block sums.  Each (head,
 // channel) sum lives in one lane and adds the bf16-rounded outputs in token
 // order, exactly as the separate pooling kernel does, so the means are
-// bit-identical to it.  The rotation of every (token, pair) of the block is
-// computed once per CTA into shared memory (while the first tokens load): a
-// warp covers 4 heads per token instead of 56, and computing the rotation per
-// warp would cost more issue slots than the HBM-bound prologue has to spare.
+// bit-identical to it.  The rotations are computed once per CTA into shared
+// memory (while the first tokens load): a pair's angle depends on one axis
+// position only, so the block needs one row of 16 (cos, sin) per distinct w,
+// per distinct (t, h) row and per distinct t of its tokens -- some 90 rows for
+// the clip grids instead of 128 tokens x 48 pairs -- and each warp steps its
+// tokens' (w, h, t) indices with counters instead of divisions.
 // Every barrier wait is bounded; an expired wait sets the device status word.
 constexpr int kPoolWarps = 7;                              // consumer warps
 constexpr int kPoolThreads = 32 * (kPoolWarps + 1);        // + the TMA producer warp
@@ -214,9 +222,13 @@ constexpr int kPoolRing = 5;                               // tokens in flight p
 constexpr int kSliceBytes = kPoolHeadsPerCta * kHeadDim * 2;  // 5,376
 static_assert(kSliceBytes % 128 == 0, "slots stay 128-byte aligned");
 
+// Rows of 16 (cos, sin) pairs the block's rotation tables can need: at most
+// 128 distinct w values plus two more rows of (t, h) for a 128-token block
+// (nw + nr <= 130 for any W), and at most 128 distinct t values.
+constexpr int kRotRows = 130 + kBlock;
 struct PoolSmem {
     uint8_t ring[kPoolRing][2][kSliceBytes];     // [slot][Q, K][28 heads x 96 bf16]
-    float2 rot[kBlock * kPairsPerHead];          // (cos, sin) per (token, pair)
+    float2 rot[kRotRows * kPairsPerSection];     // (cos, sin): w rows, then (t, h) rows, then t rows
     uint64_t full[kPoolRing], empty[kPoolRing];
     int abort_flag;
     int never;  // stays 0: abort flag for the producer's final drain
@@ -292,12 +304,25 @@ __global__ void __launch_bounds__(kPoolThreads, 2)
         return;
     }
 
-    // consumers: the block's rotations first, while the first tokens load
-    for (int e = threadIdx.x; e < len * kPairsPerHead; e += kPoolConsumers) {
-        const int i = e / kPairsPerHead, pair = e - i * kPairsPerHead;
-        const int n = n0 + i;
+    // consumers: the block's rotation tables first, while the first tokens load
+    const int HW = a.H * a.W;
+    const int w0 = n0 % a.W, r0 = n0 / a.W, t0 = n0 / HW;
+    const int nw = min(len, a.W);                       // w rows: w = (w0 + k) mod W
+    const int nr = (n0 + len - 1) / a.W - r0 + 1;       // (t, h) rows r0 .. : h = r mod H
+    const int nt = (n0 + len - 1) / HW - t0 + 1;        // t rows t0 ..
+    for (int e = threadIdx.x; e < (nw + nr + nt) * kPairsPerSection; e += kPoolConsumers) {
+        const int row = e / kPairsPerSection, j = e - row * kPairsPerSection;
+        int pos;
+        if (row < nw) {
+            pos = w0 + row;
+            if (pos >= a.W) pos -= a.W;
+        } else if (row < nw + nr) {
+            pos = (r0 + row - nw) % a.H;
+        } else {
+            pos = t0 + row - nw - nr;
+        }
         float c, sn;
-        rotation(n / (a.H * a.W), (n / a.W) % a.H, n % a.W, pair, a.freq_hi, a.freq_lo, c, sn);
+        rotation_at(pos, j, a.freq_hi, a.freq_lo, c, sn);
         sm.rot[e] = make_float2(c, sn);
     }
     asm volatile("bar.sync 1, %0;" ::"n"(kPoolConsumers) : "memory");  // the consumer warps only
@@ -319,6 +344,15 @@ __global__ void __launch_bounds__(kPoolThreads, 2)
 
     const int64_t base = static_cast<int64_t>(b) * a.sb + static_cast<int64_t>(h) * a.sh + c0;
     const int lane_off = hl * kHeadDim * 2 + sub * kChanPerLane * 2;  // byte offset of the lane's 12 channels
+    // the lane's six pairs: section (0 t, 1 h, 2 w) and index within it
+    int axis[kPairsPerLane], jj[kPairsPerLane];
+#pragma unroll
+    for (int p = 0; p < kPairsPerLane; ++p) {
+        axis[p] = (sub * kPairsPerLane + p) / kPairsPerSection;
+        jj[p] = (sub * kPairsPerLane + p) % kPairsPerSection;
+    }
+    // table rows of the current token, stepped token by token
+    int kw = 0, mh = 0, mt = 0, wcur = w0, hcur = r0 % a.H;
     bool ok = true;
     for (int t = 0; t < len; ++t) {
         const int slot = t % kPoolRing;
@@ -334,11 +368,24 @@ __global__ void __launch_bounds__(kPoolThreads, 2)
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.empty[slot]);  // the slice is in registers
         float cs[kPairsPerLane], sn[kPairsPerLane];
+        const int row_t = nw + nr + mt, row_h = nw + mh, row_w = kw;
 #pragma unroll
         for (int p = 0; p < kPairsPerLane; ++p) {
-            const float2 v = sm.rot[t * kPairsPerHead + sub * kPairsPerLane + p];
+            const int row = axis[p] == 0 ? row_t : (axis[p] == 1 ? row_h : row_w);
+            const float2 v = sm.rot[row * kPairsPerSection + jj[p]];
             cs[p] = v.x;
             sn[p] = v.y;
+        }
+        // next token: w advances; a wrap of w moves to the next (t, h) row, a
+        // wrap of h to the next t
+        if (++kw == a.W) kw = 0;
+        if (++wcur == a.W) {
+            wcur = 0;
+            ++mh;
+            if (++hcur == a.H) {
+                hcur = 0;
+                ++mt;
+            }
         }
         const int64_t off = base + static_cast<int64_t>(n0 + t) * a.sn;
         uint32_t oq[kPairsPerLane], ok_[kPairsPerLane];
