@@ -1,5 +1,5 @@
-// Packed fp32 pair arithmetic (f32x2 instructions of sm_100a) and a
-// three-input max, used by the attention softmax.
+// Packed fp32 pair arithmetic (f32x2 instructions of sm_100a), used by the
+// attention softmax and the prologue, and a three-input max.
 #pragma once
 
 #include <cstdint>
@@ -23,6 +23,11 @@ __device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
 __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
     uint64_t r;
     asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
     return r;
 }
 // max(a, b, c) in one instruction (three-input max.f32 of sm_100a).

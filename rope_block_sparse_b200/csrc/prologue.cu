@@ -17,6 +17,7 @@
 
 #include <cmath>
 
+#include "fastmath.cuh"
 #include "h3a_internal.h"
 #include "sm100.cuh"
 
@@ -51,11 +52,9 @@ struct PrologueArgs {
     uint64_t timeout_ns;  // limit of one pipeline wait
 };
 
-__device__ __forceinline__ void unpack4(uint2 v, float* x) {
-    x[0] = __uint_as_float(v.x << 16);
-    x[1] = __uint_as_float(v.x & 0xFFFF0000u);
-    x[2] = __uint_as_float(v.y << 16);
-    x[3] = __uint_as_float(v.y & 0xFFFF0000u);
+// Two packed bf16 (low half first) as an fp32 pair.
+__device__ __forceinline__ uint64_t unpack2(uint32_t v) {
+    return f2(__uint_as_float(v << 16), __uint_as_float(v & 0xFFFF0000u));
 }
 
 __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
@@ -64,29 +63,37 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
 }
 
 // Normalise, scale and rotate one lane's 12 channels of one head; out[p] holds
-// the rounded pair p as packed bf16.  Every lane of the warp must take part
-// (the RMS sum is reduced across each 8-lane group).
-__device__ __forceinline__ void norm_rope(const uint2 (&raw)[3], const float (&g)[kChanPerLane],
-                                          const float (&cs)[kPairsPerLane], const float (&sn)[kPairsPerLane],
-                                          float eps, uint32_t (&out)[kPairsPerLane]) {
-    float x[kChanPerLane];
-    unpack4(raw[0], x);
-    unpack4(raw[1], x + 4);
-    unpack4(raw[2], x + 8);
-    float ss = 0.f;
+// the rounded pair p as packed bf16.  A rotation pair (x0, x1) is one packed
+// fp32 register pair throughout: the sum of squares, the gains g2[p] = (g0, g1)
+// and the rotation rot[p] = (cos, sin) scaled by the RMS factor each take one
+// f32x2 instruction per pair.  Every lane of the warp must take part (the RMS
+// sum is reduced across each 8-lane group).
+__device__ __forceinline__ void norm_rope(const uint2 (&raw)[3], const uint64_t (&g2)[kPairsPerLane],
+                                          const uint64_t (&rot)[kPairsPerLane], float eps,
+                                          uint32_t (&out)[kPairsPerLane]) {
+    uint64_t x[kPairsPerLane];
 #pragma unroll
-    for (int i = 0; i < kChanPerLane; ++i) ss = fmaf(x[i], x[i], ss);
+    for (int q = 0; q < 3; ++q) {
+        x[2 * q] = unpack2(raw[q].x);
+        x[2 * q + 1] = unpack2(raw[q].y);
+    }
+    uint64_t ss2 = f2_mul(x[0], x[0]);
+#pragma unroll
+    for (int p = 1; p < kPairsPerLane; ++p) ss2 = f2_fma(x[p], x[p], ss2);
+    float s0, s1;
+    f2_split(ss2, s0, s1);
+    float ss = s0 + s1;
     ss += __shfl_xor_sync(0xffffffffu, ss, 1);
     ss += __shfl_xor_sync(0xffffffffu, ss, 2);
     ss += __shfl_xor_sync(0xffffffffu, ss, 4);
     const float r = rsqrtf(ss * (1.0f / kHeadDim) + eps);
+    const uint64_t r2 = f2(r, r);
 #pragma unroll
     for (int p = 0; p < kPairsPerLane; ++p) {
-        const float y0 = x[2 * p] * r * g[2 * p];
-        const float y1 = x[2 * p + 1] * r * g[2 * p + 1];
-        const float z0 = y0 * cs[p] - y1 * sn[p];
-        const float z1 = y0 * sn[p] + y1 * cs[p];
-        out[p] = pack2(z0, z1);
+        float u0, u1, c, sn;
+        f2_split(f2_mul(x[p], g2[p]), u0, u1);  // gains
+        f2_split(f2_mul(rot[p], r2), c, sn);    // rotation scaled by 1 / RMS
+        out[p] = pack2(fmaf(u0, c, -u1 * sn), fmaf(u0, sn, u1 * c));
     }
 }
 
@@ -99,12 +106,18 @@ __device__ __forceinline__ void store3(const uint32_t (&out)[kPairsPerLane], boo
     }
 }
 
-__device__ __forceinline__ void norm_rope_store(const uint2 (&raw)[3], const float (&g)[kChanPerLane],
-                                                const float (&cs)[kPairsPerLane], const float (&sn)[kPairsPerLane],
-                                                float eps, bool active, __nv_bfloat16* dst) {
+__device__ __forceinline__ void norm_rope_store(const uint2 (&raw)[3], const uint64_t (&g2)[kPairsPerLane],
+                                                const uint64_t (&rot)[kPairsPerLane], float eps, bool active,
+                                                __nv_bfloat16* dst) {
     uint32_t out[kPairsPerLane];
-    norm_rope(raw, g, cs, sn, eps, out);
+    norm_rope(raw, g2, rot, eps, out);
     store3(out, active, dst);
+}
+
+// The lane's gains as pairs (g[c0 + 2p], g[c0 + 2p + 1]).
+__device__ __forceinline__ void load_gain_pairs(const float* g, int c0, uint64_t (&g2)[kPairsPerLane]) {
+#pragma unroll
+    for (int p = 0; p < kPairsPerLane; ++p) g2[p] = f2(__ldg(g + c0 + 2 * p), __ldg(g + c0 + 2 * p + 1));
 }
 
 // cos / sin of the angle pos * theta^(-2j/32) of pair j of a section at axis
@@ -149,12 +162,9 @@ __global__ void __launch_bounds__(kThreads, 3) qk_norm_rope_kernel(const Prologu
     const int sub = lane & 7;   // 12-channel slice within the head
     const int c0 = sub * kChanPerLane;
 
-    float gq[kChanPerLane], gk[kChanPerLane];
-#pragma unroll
-    for (int i = 0; i < kChanPerLane; ++i) {
-        gq[i] = __ldg(a.gq + c0 + i);
-        gk[i] = __ldg(a.gk + c0 + i);
-    }
+    uint64_t gq[kPairsPerLane], gk[kPairsPerLane];
+    load_gain_pairs(a.gq, c0, gq);
+    load_gain_pairs(a.gk, c0, gk);
 
     const int64_t warps = static_cast<int64_t>(gridDim.x) * (kThreads / 32);
     const int head_groups = (a.heads + 3) >> 2;
@@ -165,10 +175,13 @@ __global__ void __launch_bounds__(kThreads, 3) qk_norm_rope_kernel(const Prologu
         const int pt = n / (a.H * a.W), ph = (n / a.W) % a.H, pw = n % a.W;
 
         // rotation of this lane's six pairs at this token
-        float cs[kPairsPerLane], sn[kPairsPerLane];
+        uint64_t rot[kPairsPerLane];
 #pragma unroll
-        for (int p = 0; p < kPairsPerLane; ++p)
-            rotation(pt, ph, pw, sub * kPairsPerLane + p, a.freq_hi, a.freq_lo, cs[p], sn[p]);
+        for (int p = 0; p < kPairsPerLane; ++p) {
+            float c, sn;
+            rotation(pt, ph, pw, sub * kPairsPerLane + p, a.freq_hi, a.freq_lo, c, sn);
+            rot[p] = f2(c, sn);
+        }
 
         const int64_t tok_off = static_cast<int64_t>(b) * a.sb + static_cast<int64_t>(n) * a.sn + c0;
         for (int hg = 0; hg < head_groups; hg += 2) {
@@ -181,10 +194,10 @@ __global__ void __launch_bounds__(kThreads, 3) qk_norm_rope_kernel(const Prologu
             load3(a.k + off0, act0, rk0);
             load3(a.q + off1, act1, rq1);
             load3(a.k + off1, act1, rk1);
-            norm_rope_store(rq0, gq, cs, sn, a.eps, act0, a.qo + off0);
-            norm_rope_store(rk0, gk, cs, sn, a.eps, act0, a.ko + off0);
-            norm_rope_store(rq1, gq, cs, sn, a.eps, act1, a.qo + off1);
-            norm_rope_store(rk1, gk, cs, sn, a.eps, act1, a.ko + off1);
+            norm_rope_store(rq0, gq, rot, a.eps, act0, a.qo + off0);
+            norm_rope_store(rk0, gk, rot, a.eps, act0, a.ko + off0);
+            norm_rope_store(rq1, gq, rot, a.eps, act1, a.qo + off1);
+            norm_rope_store(rk1, gk, rot, a.eps, act1, a.ko + off1);
         }
     }
 }
@@ -235,12 +248,11 @@ struct PoolSmem {
 };
 constexpr size_t kPoolSmemBytes = sizeof(PoolSmem) + 1024;  // + alignment slack
 
-__device__ __forceinline__ void add_rounded(const uint32_t (&out)[kPairsPerLane], float (&acc)[kChanPerLane]) {
+// acc[p] += the rounded pair p (one f32x2 add: the same fp32 sums, in the same
+// token order, as two scalar adds).
+__device__ __forceinline__ void add_rounded(const uint32_t (&out)[kPairsPerLane], uint64_t (&acc)[kPairsPerLane]) {
 #pragma unroll
-    for (int p = 0; p < kPairsPerLane; ++p) {
-        acc[2 * p] += __uint_as_float(out[p] << 16);
-        acc[2 * p + 1] += __uint_as_float(out[p] & 0xFFFF0000u);
-    }
+    for (int p = 0; p < kPairsPerLane; ++p) acc[p] = f2_add(acc[p], unpack2(out[p]));
 }
 
 __device__ __forceinline__ void pool_timeout(const PrologueArgs& a, volatile int* abort_flag) {
@@ -332,15 +344,12 @@ __global__ void __launch_bounds__(kPoolThreads, 2)
     const int hl = warp * 4 + (lane >> 3);  // head within the chunk
     const int h = chunk * kPoolHeadsPerCta + hl;
     const bool active = h < a.heads;
-    float gq[kChanPerLane], gk[kChanPerLane];
+    uint64_t gq[kPairsPerLane], gk[kPairsPerLane];
+    load_gain_pairs(a.gq, c0, gq);
+    load_gain_pairs(a.gk, c0, gk);
+    uint64_t accq[kPairsPerLane], acck[kPairsPerLane];
 #pragma unroll
-    for (int i = 0; i < kChanPerLane; ++i) {
-        gq[i] = __ldg(a.gq + c0 + i);
-        gk[i] = __ldg(a.gk + c0 + i);
-    }
-    float accq[kChanPerLane], acck[kChanPerLane];
-#pragma unroll
-    for (int i = 0; i < kChanPerLane; ++i) accq[i] = acck[i] = 0.f;
+    for (int p = 0; p < kPairsPerLane; ++p) accq[p] = acck[p] = f2(0.f, 0.f);
 
     const int64_t base = static_cast<int64_t>(b) * a.sb + static_cast<int64_t>(h) * a.sh + c0;
     const int lane_off = hl * kHeadDim * 2 + sub * kChanPerLane * 2;  // byte offset of the lane's 12 channels
@@ -367,14 +376,12 @@ __global__ void __launch_bounds__(kPoolThreads, 2)
         const uint2 rk[3] = {sk[0], sk[1], sk[2]};
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.empty[slot]);  // the slice is in registers
-        float cs[kPairsPerLane], sn[kPairsPerLane];
+        uint64_t rot[kPairsPerLane];
         const int row_t = nw + nr + mt, row_h = nw + mh, row_w = kw;
 #pragma unroll
         for (int p = 0; p < kPairsPerLane; ++p) {
             const int row = axis[p] == 0 ? row_t : (axis[p] == 1 ? row_h : row_w);
-            const float2 v = sm.rot[row * kPairsPerSection + jj[p]];
-            cs[p] = v.x;
-            sn[p] = v.y;
+            rot[p] = *reinterpret_cast<const uint64_t*>(&sm.rot[row * kPairsPerSection + jj[p]]);  // (cos, sin)
         }
         // next token: w advances; a wrap of w moves to the next (t, h) row, a
         // wrap of h to the next t
@@ -389,8 +396,8 @@ __global__ void __launch_bounds__(kPoolThreads, 2)
         }
         const int64_t off = base + static_cast<int64_t>(n0 + t) * a.sn;
         uint32_t oq[kPairsPerLane], ok_[kPairsPerLane];
-        norm_rope(rq, gq, cs, sn, a.eps, oq);
-        norm_rope(rk, gk, cs, sn, a.eps, ok_);
+        norm_rope(rq, gq, rot, a.eps, oq);
+        norm_rope(rk, gk, rot, a.eps, ok_);
         store3(oq, active, a.qo + off);
         store3(ok_, active, a.ko + off);
         add_rounded(oq, accq);
@@ -405,15 +412,21 @@ __global__ void __launch_bounds__(kPoolThreads, 2)
     // Q's means row-major [B, heads, nblk, 96]; K's channel-major
     // [B, heads, 96, stride], the router's layouts
     const int64_t bh = static_cast<int64_t>(b) * a.heads + h;
+    float mq[kChanPerLane], mk[kChanPerLane];
+#pragma unroll
+    for (int p = 0; p < kPairsPerLane; ++p) {
+        f2_split(accq[p], mq[2 * p], mq[2 * p + 1]);
+        f2_split(acck[p], mk[2 * p], mk[2 * p + 1]);
+    }
     float4* dq = reinterpret_cast<float4*>(a.pool_q + (bh * a.nblk + blk) * kHeadDim + c0);
 #pragma unroll
     for (int u = 0; u < kChanPerLane / 4; ++u)
-        dq[u] = make_float4(accq[4 * u] * inv_len, accq[4 * u + 1] * inv_len, accq[4 * u + 2] * inv_len,
-                            accq[4 * u + 3] * inv_len);
+        dq[u] = make_float4(mq[4 * u] * inv_len, mq[4 * u + 1] * inv_len, mq[4 * u + 2] * inv_len,
+                            mq[4 * u + 3] * inv_len);
     const int kstride = pooled_k_stride(a.nblk);
     float* dk = a.pool_k + (bh * kHeadDim + c0) * kstride + blk;
 #pragma unroll
-    for (int i = 0; i < kChanPerLane; ++i) dk[static_cast<int64_t>(i) * kstride] = acck[i] * inv_len;
+    for (int i = 0; i < kChanPerLane; ++i) dk[static_cast<int64_t>(i) * kstride] = mk[i] * inv_len;
 }
 
 // ---------------------------------------------------------------------------
