@@ -729,7 +729,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--workload", default=WORKLOAD, help="synthetic workload (clip32k: small profiler case)")
-    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--e2e-steps", type=int, default=None,
+                    help="steps of the end-to-end pass (default: --steps; 0 skips it)")
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--cpu-rows", type=int, default=4096, help="query rows of the CPU-baseline sample")
     ap.add_argument("--ref-rows", type=int, default=128, help="query rows per reference-arm step")
@@ -740,6 +741,8 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
+    if args.e2e_steps is None:
+        args.e2e_steps = args.steps
     if args.impl == "reference":
         rank = int(os.environ.get("RANK", "0"))
         world = int(os.environ.get("WORLD_SIZE", "1"))
