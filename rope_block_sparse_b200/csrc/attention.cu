@@ -13,7 +13,8 @@
 //   warps 0-7   softmax: warpgroup t = warp / 4 handles query tile t; thread r
 //               owns row r (TMEM lane r) and all 128 key columns of every
 //               block, so the row max and row sum never leave the thread.  It
-//               loads the whole row of S from TMEM with one wait, takes the
+//               loads the row of S from TMEM in two 64-column halves, taking
+//               the first half's max while the second half loads, then the
 //               block max, computes exp2 in fp32 (log2 domain, packed f32x2
 //               FMAs and adds) against the row's reference max and packs P to
 //               bf16 in place over the same registers.  The reference is fixed
@@ -459,13 +460,27 @@ __device__ void softmax_group(AttnSmem<D>& sm, const AttnArgs& a, uint32_t tmem,
         tc_fence_after_sync();
         const int kv = list ? __ldg(list + j) : j;
         const int valid = (kv == a.nblk - 1) ? a.N - kv * 128 : 128;
-        // the whole row of S in registers: one wait, the true block max before
-        // any exponential, P packed in place over the same registers
+        // the whole row of S in registers, the true block max before any
+        // exponential, P packed in place over the same registers
         uint32_t x[128];
+        float pm[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-        for (int q = 0; q < 4; ++q) tmem_ld_x32(tS + 32u * q, slice32(x + 32 * q));
+        for (int q = 0; q < 2; ++q) tmem_ld_x32(tS + 32u * q, slice32(x + 32 * q));
 #pragma unroll
-        for (int q = 0; q < 4; ++q) tmem_wait_ld_x32(slice32(x + 32 * q));
+        for (int q = 0; q < 2; ++q) tmem_wait_ld_x32(slice32(x + 32 * q));
+#pragma unroll
+        for (int q = 2; q < 4; ++q) tmem_ld_x32(tS + 32u * q, slice32(x + 32 * q));
+        // first half's max while the second half loads
+        if (valid < 64) {
+#pragma unroll
+            for (int i = 0; i < 64; ++i)
+                if (i >= valid) x[i] = __float_as_uint(-INFINITY);
+        }
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+            pm[i & 3] = max3(pm[i & 3], __uint_as_float(x[2 * i]), __uint_as_float(x[2 * i + 1]));
+#pragma unroll
+        for (int q = 2; q < 4; ++q) tmem_wait_ld_x32(slice32(x + 32 * q));
         if constexpr (kSep) {
             // S_t is in registers: release it for QK_t(j+1)
             tc_fence_before_sync();
@@ -475,12 +490,11 @@ __device__ void softmax_group(AttnSmem<D>& sm, const AttnArgs& a, uint32_t tmem,
         bool p_free = false;  // separate-P scheme: the P buffer wait is done
         if (valid < 128) {
 #pragma unroll
-            for (int i = 0; i < 128; ++i)
+            for (int i = 64; i < 128; ++i)
                 if (i >= valid) x[i] = __float_as_uint(-INFINITY);
         }
-        float pm[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-        for (int i = 0; i < 64; ++i)
+        for (int i = 32; i < 64; ++i)
             pm[i & 3] = max3(pm[i & 3], __uint_as_float(x[2 * i]), __uint_as_float(x[2 * i + 1]));
         const float mx = c * fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3]));
         if (j == 0) {
