@@ -156,7 +156,10 @@ __device__ __forceinline__ void load3(const __nv_bfloat16* src, bool active, uin
     }
 }
 
-__global__ void __launch_bounds__(kThreads, 3) qk_norm_rope_kernel(const PrologueArgs a) {
+// Two CTAs per SM: the 128 registers that allows hold two head groups' loads
+// of Q and K without spilling (at three CTAs, 80 registers, the kernel
+// spilled and ran 5% slower).
+__global__ void __launch_bounds__(kThreads, 2) qk_norm_rope_kernel(const PrologueArgs a) {
     const int lane = threadIdx.x & 31;
     const int grp = lane >> 3;  // head within a group of four
     const int sub = lane & 7;   // 12-channel slice within the head
