@@ -737,7 +737,7 @@ def run_reference(args, rank, world):
     }
 
 
-def main():
+def parse_args(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=10)
@@ -753,11 +753,16 @@ def main():
                     help="skip the 245,952-token pass reported beside the headline")
     ap.add_argument("--kernel-only", choices=["router"], default=None,
                     help="time one kernel alone on a small case for profilers (one GPU): router = scores + top-k")
-    args = ap.parse_args()
+    args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     if args.e2e_steps is None:
         args.e2e_steps = args.steps
+    return args
+
+
+def main():
+    args = parse_args()
     if args.impl == "reference":
         rank = int(os.environ.get("RANK", "0"))
         world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -70,3 +70,9 @@ def test_reference_arm_under_torchrun_prints_once():
     assert len(lines) == 1, res.stdout
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["config"]["parallelism"].startswith("dp2")
+
+
+def test_end_to_end_pass_runs_the_timed_step_count_unless_told_otherwise():
+    assert bench.parse_args(["--steps", "20", "--warmup", "3"]).e2e_steps == 20
+    assert bench.parse_args([]).e2e_steps == bench.parse_args([]).steps
+    assert bench.parse_args(["--steps", "7", "--e2e-steps", "0"]).e2e_steps == 0
