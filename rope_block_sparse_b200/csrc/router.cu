@@ -9,12 +9,14 @@
 //                       block's 128 token rows (all heads) once and writes fp32
 //                       means: Q's [B, heads, nblk, D], K's channel-major
 //                       [B, heads, D, nblk rounded up to 4].
-//   score_topk_kernel   one CTA per (batch*head, 16 query blocks): fp32 scores of
+//   score_topk_kernel   one CTA per (batch*head, 8 query blocks): fp32 scores of
 //                       its query blocks against every key block into shared
 //                       memory (8 x 4 register tiles over the channel-major K
 //                       means), then one warp per query block selects the top k
-//                       with a 4-pass 8-bit radix select over order-preserving
-//                       32-bit keys and emits the indices in ascending order.
+//                       -- 256 buckets linear in the score and an exact ranking
+//                       of the bucket holding the cut, or a 4-pass 8-bit radix
+//                       select over order-preserving 32-bit keys when that
+//                       bucket is crowded -- and emits the indices ascending.
 #include <cuda_bf16.h>
 
 #include <cmath>
@@ -28,8 +30,15 @@ constexpr int kPoolThreads = 224;    // 672 16-byte vectors per CTA row: 56 head
 constexpr int kVecPerThread = 3;
 template <int D>
 constexpr int heads_per_pool_cta() { return kPoolThreads * kVecPerThread / (D / 8); }
-constexpr int kScoreThreads = 512;   // 16 warps
-constexpr int kRowsPerCta = 16;      // query blocks per score CTA (one warp each)
+// Eight query blocks per score CTA (one warp each in the selection), four
+// CTAs per SM: half-size CTAs keep more of them resident at large nblk and
+// overlap one CTA's scores with another's selection (16-block CTAs, two per
+// SM, took 0.444 against 0.413 ms at 977 blocks and 2.28 against 1.74 ms at
+// 1,922, with identical lists).
+constexpr int kScoreThreads = 256;   // 8 warps
+constexpr int kRowsPerCta = 8;       // query blocks per score CTA
+static_assert(kScoreThreads / 256 * 8 == kRowsPerCta && kScoreThreads / 32 == kRowsPerCta,
+              "8 x 4 score tiles over 256 key groups; one selecting warp per query block");
 constexpr int kScoreSmemLimit = 200 * 1024;
 
 struct PoolArgs {
@@ -175,23 +184,23 @@ __device__ __forceinline__ void select_digit(const uint32_t* h, int lane, uint32
     above = __shfl_sync(0xffffffffu, ab, src);
 }
 
-// grid: (ceil(nblk / 16), B*heads), 512 threads.  Dynamic shared memory:
-// qbar[D][16] fp32 (the CTA's 16 query-block means, channel-major),
-// scores[16][nblk4] fp32 (nblk4 = nblk rounded up to 4), histograms[16][256] u32.
+// grid: (ceil(nblk / 8), B*heads), 256 threads.  Dynamic shared memory:
+// qbar[D][8] fp32 (the CTA's 8 query-block means, channel-major),
+// scores[8][nblk4] fp32 (nblk4 = nblk rounded up to 4), histograms[8][256] u32.
 //
-// Scores: thread t computes query blocks 8*(t/256) .. +7 against key blocks
-// j0 + 4*(t%256) .. +3, j0 = 0, 1024, ...: an 8 x 4 register tile.  Per
+// Scores: thread t computes the CTA's 8 query blocks against key blocks
+// j0 + 4*t .. +3, j0 = 0, 1024, ...: an 8 x 4 register tile.  Per
 // channel it reads its four key means with one 16-byte load -- the K means are
 // channel-major, so a warp's loads are 512 contiguous bytes -- and two 16-byte
 // broadcasts of the query means.  Every dot product adds q_c * k_c in channel
 // order c = 0..D-1 with one fmaf per channel, then scales by 1/sqrt(D).
 template <int D>
-__global__ void __launch_bounds__(kScoreThreads, 2) score_topk_kernel(const ScoreArgs a) {
+__global__ void __launch_bounds__(kScoreThreads, 4) score_topk_kernel(const ScoreArgs a) {
     extern __shared__ __align__(16) float smem[];
     const int nblk4 = pooled_k_stride(a.nblk);
-    float* qbar = smem;                                                  // [D][16]
-    float* scores = qbar + kRowsPerCta * D;                              // [16][nblk4]
-    uint32_t* hist = reinterpret_cast<uint32_t*>(scores + kRowsPerCta * nblk4);  // [16][256]
+    float* qbar = smem;                                                  // [D][8]
+    float* scores = qbar + kRowsPerCta * D;                              // [8][nblk4]
+    uint32_t* hist = reinterpret_cast<uint32_t*>(scores + kRowsPerCta * nblk4);  // [8][256]
 
     const int bh = blockIdx.y;
     const int i0 = blockIdx.x * kRowsPerCta;
