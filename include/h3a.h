@@ -133,8 +133,12 @@ h3a_status h3a_route_workspace_size(const h3a_qkv_desc* d, int32_t block, size_t
  * k_out      : host; receives k (may be NULL).
  * workspace  : device, at least h3a_route_workspace_size bytes, 16-B aligned.
  * Errors: INVALID_ARG for null pointers or sparsity outside [0, 1);
- * UNSUPPORTED for block != 128 or head_dim other than 96 / 128; WORKSPACE if
- * the workspace is null or ws_bytes is too small. */
+ * UNSUPPORTED for block != 128, head_dim other than 96 / 128, more key blocks
+ * than the score kernel holds (each of its CTAs keeps 8 query blocks' fp32
+ * scores against every key block in 200 KB of shared memory: ceil(N / 128)
+ * <= 6,048 at head_dim 96, 6,016 at 128) or B * heads > 65,535; WORKSPACE if
+ * the workspace is null or ws_bytes is too small.  Nothing is launched when a
+ * check fails. */
 h3a_status h3a_route(const void* q, const void* k, const h3a_qkv_desc* d, double sparsity,
                      int32_t block, int32_t* block_idx, int64_t* k_out, void* workspace,
                      size_t ws_bytes, h3a_stream_t stream);

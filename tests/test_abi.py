@@ -120,6 +120,13 @@ def test_route_validation():
     assert call(w=None) == 5
     assert call(wsb=ws - 1) == 5
     assert call(w=MISALIGNED) == 5
+    # the score kernel keeps a CTA's 8 query-block rows of fp32 scores against
+    # every key block in shared memory: 6,048 key blocks at head_dim 96 and
+    # 6,016 at 128 (200 KB); past that the call is refused before any launch
+    for D, most in ((96, 6048), (128, 6016)):
+        assert call(desc=_desc(N=most * 128, heads=1, D=D), wsb=0) == 5      # shape accepted, workspace short
+        assert call(desc=_desc(N=most * 128 + 1, heads=1, D=D), wsb=0) == 2
+    assert call(desc=_desc(B=65536, N=128, heads=1)) == 2                  # B * heads beyond the grid's y range
 
 
 @NO_GPU
